@@ -1,0 +1,468 @@
+"""Benchmark: fused split-KV GQA decode attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one call of the fused decode (every step of the path: split
+assignment, TMA-fed K/V stream, logits, online softmax, PV, triplets and the
+log-sum-exp merge) over one batch of the workload, inputs resident in HBM.
+Metric (the headline of the method's target): KV bytes read per second
+(GB/s), with us/call and the fraction of measured HBM bandwidth.  Between
+timed steps the inputs rotate among copies totalling >= 1 GiB so no step
+reads K/V from L2.  Multi-GPU runs are independent replicas (one per rank,
+weak scaling); time is the max over ranks of CUDA-event time.
+
+--impl reference times the CPU oracle (fp64, every host core) on a bounded
+sample of the same workload per step; the GPU is not used.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "GQA decode attention: KV-read HBM GB/s and % of B200 peak; µs/call"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+ROTATE_TOTAL = 1 << 30
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_tc_bf16_llama70b.md")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20000)
+    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--config", default="llama70b", choices=sorted(workloads.CONFIGS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------- helpers
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gqa_split_kv_decode_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources and this workload (else None)."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    src = re.search(r"kernel_source_hash:\s*(\w+)", text)
+    wl = re.search(r"workload:\s*(\w+)", text)
+    tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (src and wl and tr) or src.group(1) != kernel_source_hash() or wl.group(1) != config:
+        return None
+    return int(tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.lines:
+            return None
+        window = [l for (t, l) in self.lines if self.t0 is not None and self.t0 - 0.1 <= t <= (self.t1 or t) + 0.1]
+        rows = window or [l for _, l in self.lines]
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [x.strip() for x in r.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "in_window": bool(window)}
+
+
+# ----------------------------------------------------------------- our arm
+
+def workload_desc(c) -> str:
+    if c.chunk_len:
+        split = f"chunk_len={c.chunk_len}, S_b~U[{c.S_min},{c.S}]"
+    else:
+        split = f"S={c.S}, n_splits={c.n_splits}"
+    return (f"{c.name}: B={c.B}, h_q={c.h_q}, h_kv={c.h_kv}, d_head={c.d}, {split}, "
+            f"{c.dtype} q/k/v, fp32 out")
+
+
+def run_ours(args, rank, world, local_rank):
+    import gqa_split_kv_decode_b200 as gk
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    cfg = workloads.CONFIGS[args.config]
+    w = workloads.generate(cfg)
+    kv_bytes = w.kv_bytes
+    n_copies = max(1, math.ceil(ROTATE_TOTAL / kv_bytes)) if kv_bytes < 2 * L2_BYTES else 1
+    q = w.q.to(device)
+    sl = w.seqlens.to(device)
+    ks = [w.k.to(device) for _ in range(n_copies)]
+    vs = [w.v.to(device) for _ in range(n_copies)]
+    out = torch.empty((cfg.B, cfg.h_q, cfg.d), dtype=torch.float32, device=device)
+    if cfg.chunk_len:
+        ws = torch.zeros(gk.chunked_workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.chunk_len,
+                                                   w.max_seqlen), dtype=torch.uint8, device=device)
+        call = lambda i: gk.gqa_decode_attn_chunked(q, ks[i % n_copies], vs[i % n_copies], sl,
+                                                    cfg.chunk_len, w.max_seqlen, cfg.scale, out=out,
+                                                    workspace=ws)
+    else:
+        ws = torch.zeros(gk.workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.n_splits),
+                         dtype=torch.uint8, device=device)
+        call = lambda i: gk.gqa_decode_attn(q, ks[i % n_copies], vs[i % n_copies], sl, cfg.n_splits,
+                                            cfg.scale, out=out, workspace=ws)
+    stream = torch.cuda.current_stream(device)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize(device)
+    if gk.get_status(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
+        time.sleep(0.6)  # let the sampler start before the timed region
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_begin()
+    for i in range(K):
+        starts[i].record(stream)
+        call(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    if world > 1:
+        dist.barrier()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    per_launch_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+    status = gk.get_status(device)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    sampler.stop()
+    clocks = sampler.summary() if rank == 0 else None
+
+    max_total_ms = max_over_ranks(total_ms, world, device)
+    max_launch_ms = max_over_ranks(per_launch_ms, world, device)
+    all_bytes = sum_over_ranks(float(kv_bytes) * K, world, device)
+
+    # ---- end to end through the public API: pinned host inputs in, result out
+    E = max(1, min(args.e2e_steps, K))
+    hq = w.q.pin_memory()
+    hk = w.k.pin_memory()
+    hv = w.v.pin_memory()
+    hsl = w.seqlens.pin_memory()
+    hout = torch.empty_like(out, device="cpu").pin_memory()
+    dq, dk, dv, dsl = torch.empty_like(q), torch.empty_like(ks[0]), torch.empty_like(vs[0]), torch.empty_like(sl)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        if cfg.chunk_len:
+            gk.gqa_decode_attn_chunked(dq, dk, dv, dsl, cfg.chunk_len, w.max_seqlen, cfg.scale, out=out,
+                                       workspace=ws)
+        else:
+            gk.gqa_decode_attn(dq, dk, dv, dsl, cfg.n_splits, cfg.scale, out=out, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, device)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl))
+    d2h = hout.numel() * hout.element_size()
+    e2e_bytes = sum_over_ranks(float(kv_bytes), world, device)
+
+    if rank != 0:
+        return None
+
+    peak, peak_src = measured_hbm_peak()
+    ms_per_step = max_total_ms / K
+    value = all_bytes / (max_total_ms * 1e-3) / 1e9
+    achieved = kv_bytes / (max_launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6),
+        "us_per_call": round(ms_per_step * 1e3, 3),
+        "pct_of_hbm_peak": round(100.0 * value / (peak * world), 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
+        "config": {
+            "workload": workload_desc(cfg),
+            "kv_bytes_per_step": kv_bytes,
+            "global_batch": cfg.B * world,
+            "seq_len": cfg.S,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": (f"K/V rotate among {n_copies} copies ({n_copies * kv_bytes / 2**30:.2f} GiB); "
+                   f"each step's K/V ({kv_bytes / 2**20:.0f} MiB) "
+                   + ("exceeds" if kv_bytes > L2_BYTES else "is below") + " the 126 MB L2"),
+            "accumulate": "fp32 (bf16 tensor-core products, fp32 softmax and merge)",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured" else "fallback",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(cfg.name),
+            "algorithmic_bytes_per_launch": kv_bytes,
+            "kernel": "decode_tc_bf16 (fused, one launch per step)" if cfg.dtype == "bf16" else "decode_simt_f32",
+            "launch_ms": round(max_launch_ms, 6),
+        },
+        "e2e": {
+            "value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 3),
+            "unit": UNIT,
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(e2e_ms, 4),
+            "note": "pinned host q/k/v/seqlens copied in and out copied back every step",
+        },
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
+    return line
+
+
+# ------------------------------------------------------- the CPU oracle arm
+
+def oracle_sample(w, n_items: int, start: int):
+    """n_items (b, h) pairs of the workload, cycling through all of them."""
+    c = w.cfg
+    total = c.B * c.h_q
+    idx = [(start + i) % total for i in range(n_items)]
+    return [(i // c.h_q, i % c.h_q) for i in idx]
+
+
+def cpu_baseline(w, budget_s: float):
+    """Times the oracle as it stands on a sample of (b, h) rows; KV GB/s is
+    the workload's KV bytes scaled by the sampled fraction of its rows."""
+    import oracle
+    c = w.cfg
+    total = c.B * c.h_q
+    cores = os.cpu_count() or 1
+    n = min(total, max(cores, 1))
+    t0 = time.perf_counter()
+    oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=oracle_sample(w, n, 0))
+    dt = time.perf_counter() - t0
+    per_item = dt / n
+    n_run = int(min(total * 4, max(n, budget_s / max(per_item, 1e-9))))
+    t0 = time.perf_counter()
+    done, start = 0, n
+    while done < n_run:
+        m = min(total, n_run - done)
+        oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=oracle_sample(w, m, start))
+        start += m
+        done += m
+    dt = time.perf_counter() - t0
+    kv_equiv = w.kv_bytes * done / total
+    return {"value": round(kv_equiv / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} of the workload's {total} (b, h) output rows (fp64 two-pass, "
+                      f"{dt:.1f} s); KV bytes scaled by the sampled fraction",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    cfg = workloads.CONFIGS[args.config]
+    w = workloads.generate(cfg)
+    c = w.cfg
+    total = c.B * c.h_q
+    cores = os.cpu_count() or 1
+    # size each step so the whole run stays near two minutes
+    t0 = time.perf_counter()
+    oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=oracle_sample(w, cores, 0))
+    per_item = (time.perf_counter() - t0) / cores
+    steps = args.steps + args.warmup
+    n_items = int(max(1, min(total, 120.0 / max(steps, 1) / max(per_item, 1e-9))))
+    for i in range(args.warmup):
+        oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=oracle_sample(w, n_items, i * n_items))
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale,
+                    items=oracle_sample(w, n_items, (args.warmup + i) * n_items))
+    dt = time.perf_counter() - t0
+    kv_equiv = w.kv_bytes * n_items / total * args.steps
+    value = kv_equiv / dt / 1e9
+    sample = f"{n_items} of {total} (b, h) output rows per step; KV bytes scaled by that fraction"
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(1, args.steps), 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same workload as the GPU arm)",
+        "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local_rank = dist_env()
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,248 @@
+"""Grouped-query split-KV decode attention for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libgqadecode.so`` (C ABI in ``include/gqa_decode.h``).
+PyTorch is used for device memory and the current stream only: every step of
+the computation runs in the library's CUDA kernels.  If the library is
+missing, importing this package raises ImportError -- there is no fallback.
+
+Layouts (see the header): q [B, h_q, d]; k_cache, v_cache packed
+[sum S_b, h_kv, d]; seqlens int32 [B] on the device; out fp32 [B, h_q, d];
+triplets m, l [B, h_q, n_slots] and o [B, h_q, n_slots, d] in fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "gqa_decode_attn", "gqa_decode_attn_chunked", "gqa_decode_partial",
+    "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
+    "get_status", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "GQADecodeError", "LIB_PATH", "F32", "BF16",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqadecode.so")
+F32, BF16 = 0, 1
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE_TIMEOUT, ERR_DEVICE_SEQLEN = range(7)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m gqa_split_kv_decode_b200._build` "
+        "(nvcc, sm_100a). There is no CPU or eager fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _sz, _ci, _cf, _ull = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong
+
+
+def _sig(name, res, *args):
+    fn = getattr(_lib, name)
+    fn.restype = res
+    fn.argtypes = list(args)
+    return fn
+
+
+_version = _sig("gqa_decode_version", _ci)
+_errstr = _sig("gqa_decode_error_string", ctypes.c_char_p, _ci)
+_ws_size = _sig("gqa_decode_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci)
+_ws_size_chunked = _sig("gqa_decode_chunked_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci, _ci)
+_attn = _sig("gqa_decode_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _ci,
+             _vp, _sz, _vp)
+_attn_chunked = _sig("gqa_decode_attn_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
+                     _ci, _ci, _cf, _ci, _vp, _sz, _vp)
+_partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
+                _ci, _cf, _ci, _vp)
+_partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci,
+                        _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
+_merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
+_get_status = _sig("gqa_decode_get_status", _ci, _vp)
+_set_timeout = _sig("gqa_decode_set_wait_timeout_ns", _ci, _ull)
+_selftest = _sig("gqa_decode_selftest_wait_timeout", _ci, _ull, _vp)
+_release = _sig("gqa_decode_release", _ci)
+
+
+class GQADecodeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_errstr(status).decode()}")
+
+
+def _check(rc: int, where: str):
+    if rc != OK:
+        raise GQADecodeError(rc, where)
+
+
+def version() -> int:
+    return _version()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q/k/v must be bf16 or fp32, got {t.dtype}")
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _inputs(q, k_cache, v_cache, seqlens):
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("seqlens", seqlens)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.device == k_cache.device == v_cache.device == seqlens.device):
+        raise ValueError("all tensors must be on one device")
+    if q.dim() != 3 or k_cache.dim() != 3 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [B, h_q, d]; k_cache, v_cache [rows, h_kv, d]")
+    if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
+        raise ValueError("q, k_cache and v_cache must share one dtype")
+    if seqlens.dtype != torch.int32 or seqlens.dim() != 1 or seqlens.shape[0] != q.shape[0]:
+        raise ValueError("seqlens must be int32 [B]")
+    if q.shape[2] != k_cache.shape[2]:
+        raise ValueError("head dims differ")
+    B, h_q, d = q.shape
+    return B, h_q, k_cache.shape[1], d, _dtype_code(q)
+
+
+def _default_scale(d: int, scale):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+_workspaces: dict = {}
+
+
+def _workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    """Grow-only zero-filled workspace per device, owned by torch's allocator."""
+    key = (device.type, device.index)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def _out(out, shape, device):
+    if out is None:
+        return torch.empty(shape, dtype=torch.float32, device=device)
+    if out.dtype != torch.float32 or tuple(out.shape) != tuple(shape) or not out.is_contiguous():
+        raise ValueError(f"out must be contiguous fp32 {tuple(shape)}")
+    if out.device != device:
+        raise ValueError("out must be on the inputs' device")
+    return out
+
+
+def workspace_size(B, h_q, h_kv, d, n_splits) -> int:
+    return _ws_size(B, h_q, h_kv, d, n_splits)
+
+
+def chunked_workspace_size(B, h_q, h_kv, d, chunk_len, max_seqlen) -> int:
+    return _ws_size_chunked(B, h_q, h_kv, d, chunk_len, max_seqlen)
+
+
+def gqa_decode_attn(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, out=None,
+                    workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused split-KV decode attention (split by count); returns fp32 [B, h_q, d]."""
+    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out(out, (B, h_q, d), q.device)
+    need = _ws_size(B, h_q, h_kv, d, n_splits)
+    if workspace is None:
+        workspace = _workspace(q.device, need)
+    with torch.cuda.device(q.device):
+        _check(_attn(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                     out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
+                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                     _stream(q.device)), "gqa_decode_attn")
+    return out
+
+
+def gqa_decode_attn_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_seqlen: int,
+                            scale=None, out=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused split-KV decode attention with fixed chunks (ragged batches)."""
+    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out(out, (B, h_q, d), q.device)
+    need = _ws_size_chunked(B, h_q, h_kv, d, chunk_len, max_seqlen)
+    if workspace is None:
+        workspace = _workspace(q.device, need)
+    with torch.cuda.device(q.device):
+        _check(_attn_chunked(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                             out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
+                             _default_scale(d, scale), dt, workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(q.device)),
+               "gqa_decode_attn_chunked")
+    return out
+
+
+def _triplets(B, h_q, n, d, device, m, l, o):
+    m = _out(m, (B, h_q, n), device)
+    l = _out(l, (B, h_q, n), device)
+    o = _out(o, (B, h_q, n, d), device)
+    return m, l, o
+
+
+def gqa_decode_partial(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, m=None, l=None, o=None):
+    """Per-split (m, l, o) triplets (split by count)."""
+    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    m, l, o = _triplets(B, h_q, n_splits, d, q.device, m, l, o)
+    with torch.cuda.device(q.device):
+        _check(_partial(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+                        m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
+                        _default_scale(d, scale), dt, _stream(q.device)), "gqa_decode_partial")
+    return m, l, o
+
+
+def gqa_decode_partial_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_seqlen: int,
+                               scale=None, m=None, l=None, o=None):
+    """Per-chunk (m, l, o) triplets; n_slots = max(1, ceil(max_seqlen / chunk_len))."""
+    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    n = max(1, -(-max_seqlen // chunk_len)) if chunk_len > 0 and max_seqlen >= 0 else 1
+    m, l, o = _triplets(B, h_q, n, d, q.device, m, l, o)
+    with torch.cuda.device(q.device):
+        _check(_partial_chunked(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                seqlens.data_ptr(), m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q,
+                                h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
+                                _stream(q.device)), "gqa_decode_partial_chunked")
+    return m, l, o
+
+
+def mlo_merge(m, l, o, out=None) -> torch.Tensor:
+    """Log-sum-exp merge + normalisation of [..., n] triplets -> fp32 [..., d]."""
+    for name, t in (("m", m), ("l", l), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    n, d = o.shape[-2], o.shape[-1]
+    lead = tuple(m.shape[:-1])
+    if tuple(m.shape) != lead + (n,) or tuple(l.shape) != lead + (n,) or tuple(o.shape) != lead + (n, d):
+        raise ValueError("shapes: m, l [..., n]; o [..., n, d]")
+    rows = int(math.prod(lead))
+    out = _out(out, lead + (d,), m.device)
+    with torch.cuda.device(m.device):
+        _check(_merge(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
+                      _stream(m.device)), "mlo_merge")
+    return out
+
+
+def get_status(device=None) -> int:
+    """Synchronise the current stream, read and clear the device status word."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        return _get_status(_stream(device))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _check(_set_timeout(ns), "gqa_decode_set_wait_timeout_ns")
+
+
+def selftest_wait_timeout(ns: int, device=None) -> None:
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        _check(_selftest(ns, _stream(device)), "gqa_decode_selftest_wait_timeout")
+
+
+def release() -> None:
+    _check(_release(), "gqa_decode_release")

@@ -1,0 +1,99 @@
+// fp32 decode attention on the CUDA cores.
+//
+// fp32 inputs must not go through TF32 or bf16 tensor-core products (the fp32
+// tolerance is 1e-5), so this path uses plain FMA.  It serves the small fp32
+// workloads, which are launch-bound: a warp streams one key row per step with
+// 16-byte (D = 128) or 8-byte (D = 64) loads per lane, all HB query heads of
+// the block reuse that row, and the online softmax is kept per warp in base 2.
+#pragma once
+
+#include "split_merge.cuh"
+
+namespace gqa {
+
+template <int D, int HB, int NW, int MODE>
+__global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
+  static_assert(D == 64 || D == 128, "head dim");
+  constexpr int PER = D / 32;  // contiguous elements per lane
+  __shared__ float sm_m[NW * HB], sm_l[NW * HB];
+  __shared__ __align__(16) float sm_o[NW * HB * D];
+  __shared__ int sm_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = blockIdx.x, b = blockIdx.z;
+  const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
+  const Split sp = locate_split(a, b, slot, lane,
+                                warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
+  if (slot >= sp.n_active) {
+    if (MODE == kPartial) emit_empty_triplet<HB, D>(a, b, g, hb, slot);
+    return;
+  }
+
+  const float* __restrict__ qp = static_cast<const float*>(a.q);
+  const float* __restrict__ kp = static_cast<const float*>(a.k);
+  const float* __restrict__ vp = static_cast<const float*>(a.v);
+
+  float qr[HB][PER];
+#pragma unroll
+  for (int hh = 0; hh < HB; ++hh) {
+    const int gi = hb * HB + hh;
+    const float* src = qp + query_row(a, b, g, gi < a.G ? gi : 0) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) qr[hh][e] = gi < a.G ? src[e] : 0.f;
+  }
+
+  float m_run[HB], l_run[HB], o_acc[HB][PER];
+#pragma unroll
+  for (int hh = 0; hh < HB; ++hh) {
+    m_run[hh] = -INFINITY;
+    l_run[hh] = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) o_acc[hh][e] = 0.f;
+  }
+
+  for (int j = sp.lo + warp; j < sp.hi; j += NW) {
+    const size_t base = ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
+    float kr[PER], vr[PER];
+    if constexpr (PER == 4) {
+      const float4 k4 = __ldg(reinterpret_cast<const float4*>(kp + base));
+      const float4 v4 = __ldg(reinterpret_cast<const float4*>(vp + base));
+      kr[0] = k4.x; kr[1] = k4.y; kr[2] = k4.z; kr[3] = k4.w;
+      vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
+    } else {
+      const float2 k2 = __ldg(reinterpret_cast<const float2*>(kp + base));
+      const float2 v2 = __ldg(reinterpret_cast<const float2*>(vp + base));
+      kr[0] = k2.x; kr[1] = k2.y;
+      vr[0] = v2.x; vr[1] = v2.y;
+    }
+#pragma unroll
+    for (int hh = 0; hh < HB; ++hh) {
+      if (hb * HB + hh >= a.G) break;
+      float part = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) part = fmaf(qr[hh][e], kr[e], part);
+      const float s = warp_sum(part) * a.scale_log2;
+      const float m_new = fmaxf(m_run[hh], s);
+      const float alpha = exp2f(m_run[hh] - m_new);  // 0 on the first key
+      const float p = exp2f(s - m_new);
+      l_run[hh] = fmaf(l_run[hh], alpha, p);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o_acc[hh][e] = fmaf(o_acc[hh][e], alpha, p * vr[e]);
+      m_run[hh] = m_new;
+    }
+  }
+
+#pragma unroll
+  for (int hh = 0; hh < HB; ++hh) {
+    if (lane == 0) {
+      sm_m[warp * HB + hh] = m_run[hh];
+      sm_l[warp * HB + hh] = l_run[hh];
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) sm_o[(warp * HB + hh) * D + lane * PER + e] = o_acc[hh][e];
+  }
+  __syncthreads();
+  emit_split_triplet<NW, HB, D>(sm_m, sm_l, sm_o, a, b, g, hb, slot);
+  if (MODE == kFused) fused_finish<NW, HB, D>(a, b, g, hb, sp.n_active, &sm_flag);
+}
+
+}  // namespace gqa

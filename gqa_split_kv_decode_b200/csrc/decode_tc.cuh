@@ -1,0 +1,306 @@
+// bf16 decode attention: TMA-fed K/V tiles, tensor-core logits and PV.
+//
+// One CTA owns one (split, kv head g, head block, b).  Each of its NW warps
+// runs its own NS-stage TMA ring: a stage holds KT = 16 consecutive keys of K
+// and V for kv head g (one 64-element, 128-byte-swizzled box per half of
+// d_head), loaded once from HBM and shared by every query head of the group
+// (exllama "Llama 2 is out": broadcast the kv head to its group instead of
+// copying the cache).  Warp w takes the split's tiles w, w + NW, ..., so the
+// warps of a CTA are sub-splits whose triplets are merged in shared memory at
+// the end -- the page's merge rule once more.
+//
+// The products are oriented so the group, not the keys, is the narrow side:
+//   S^T[key][head] = K[key][:] . Q^T[:][head]     mma m16n8k16, M = 16 keys,
+//                                                 N = 8 heads, K = d
+//   o^T[d][head]  += V^T[d][key] . P^T[key][head] M = 16 dims, N = 8 heads,
+//                                                 K = 16 keys
+// so a group of 8 (Llama-70B) fills N exactly.  Q^T stays in registers for
+// the whole split; the S^T accumulator becomes P^T's B fragment through one
+// movmatrix transpose per 8x8 block.  Softmax statistics are fp32 in base 2
+// (scale * log2 e is folded into one multiply), reduced with shuffles across
+// the 8 lanes that share a head.  P is rounded to bf16 for the PV product and
+// the denominator sums those same rounded weights.
+//
+// The last tile of a split that is not a whole tile is loaded as the KT rows
+// that END at the split's end (shifted back) and the rows before the tile's
+// first new key are masked by index, so no load ever reaches past the
+// batch's last cache row.  A shift below row 0 reads TMA zero fill.
+#pragma once
+
+#include "split_merge.cuh"
+
+namespace gqa {
+
+constexpr int kTileKeys = 16;
+constexpr int kBoxBytes = kTileKeys * 128;  // 16 rows x 64 bf16 (one d half)
+
+template <int D>
+struct TcShape {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kStageBytes = 2 * kHalves * kBoxBytes;  // K halves, then V halves
+  static constexpr int kSteps = D / 16;                        // k-steps of S^T, d-tiles of o^T
+};
+
+template <int D, int NW, int NS>
+constexpr int tc_dynamic_smem() {
+  return NW * NS * TcShape<D>::kStageBytes + 1024;  // + slack for 1024-byte alignment
+}
+
+template <int D, int NT, int NW, int NS, int MODE>
+__global__ void __launch_bounds__(NW * 32)
+    decode_tc_bf16(const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(NT == 1 || NT == 2, "heads per CTA: 8 or 16");
+  constexpr int HB = NT * 8;
+  constexpr int KT = kTileKeys;
+  constexpr int HALVES = TcShape<D>::kHalves;
+  constexpr int STAGE = TcShape<D>::kStageBytes;
+  constexpr int STEPS = TcShape<D>::kSteps;
+  static_assert(HB * D * 4 <= NS * STAGE, "per-warp o staging must fit in the warp's stages");
+
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[NW * NS];
+  __shared__ float sm_m[NW * HB], sm_l[NW * HB];
+  __shared__ int sm_flag;
+
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = blockIdx.x, b = blockIdx.z;
+  const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
+  const Split sp = locate_split(a, b, slot, lane,
+                                warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
+  if (slot >= sp.n_active) {
+    if (MODE == kPartial) emit_empty_triplet<HB, D>(a, b, g, hb, slot);
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+#pragma unroll
+    for (int i = 0; i < NW * NS; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // Q^T as the B operand of S^T = K Q^T: thread holds head (lane / 4) and
+  // d = 16 * ks + 2 * (lane % 4) + {0, 1} (b0) and + {8, 9} (b1).
+  uint32_t qf[NT][STEPS][2];
+  {
+    const uint32_t* qw = static_cast<const uint32_t*>(a.q);  // bf16 pairs
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int gi = hb * HB + nt * 8 + (lane >> 2);
+      const bool ok = gi < a.G;
+      const size_t base = (query_row(a, b, g, ok ? gi : 0) * D) / 2 + (lane & 3);
+#pragma unroll
+      for (int ks = 0; ks < STEPS; ++ks) {
+        qf[nt][ks][0] = ok ? __ldg(qw + base + ks * 8) : 0u;
+        qf[nt][ks][1] = ok ? __ldg(qw + base + ks * 8 + 4) : 0u;
+      }
+    }
+  }
+
+  const int len = sp.hi - sp.lo;
+  const int ntiles = (len + KT - 1) / KT;
+  const uint64_t policy = l2_policy_evict_first();
+  const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
+  const uint32_t bar0 = smem_u32(&full_bar[warp * NS]);
+
+  // First row (relative to the sequence) that tile t loads.
+  auto tile_row0 = [&](int t) {
+    const int ts = sp.lo + t * KT;
+    return (ts + KT <= sp.hi) ? ts : sp.hi - KT;
+  };
+  auto issue = [&](int t, int s) {
+    const uint32_t bar = bar0 + s * 8;
+    const uint32_t dst = stage0 + s * STAGE;
+    const int row = static_cast<int>(sp.off + tile_row0(t));
+    mbar_arrive_expect_tx(bar, STAGE);
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) tma_load_3d(dst + h * kBoxBytes, &kmap, h * 64, g, row, bar, policy);
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h)
+      tma_load_3d(dst + (HALVES + h) * kBoxBytes, &vmap, h * 64, g, row, bar, policy);
+  };
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int t = warp + s * NW;
+      if (t < ntiles) issue(t, s);
+    }
+  }
+  __syncwarp();
+
+  float m_run[NT][2], l_run[NT][2];
+  float oacc[STEPS][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oacc[dt][nt][e] = 0.f;
+  }
+
+  int it = 0;
+  bool failed = false;
+  for (int t = warp; t < ntiles; t += NW, ++it) {
+    const int s = it % NS;
+    const uint32_t parity = (it / NS) & 1;
+    const bool ok = mbar_wait_bounded(bar0 + s * 8, parity, a.timeout_ns);
+    if (!__all_sync(kFull, ok)) {
+      failed = true;
+      break;
+    }
+    const uint32_t kbase = stage0 + s * STAGE;
+    const uint32_t vbase = kbase + HALVES * kBoxBytes;
+
+    // ---- S^T = K Q^T (16 keys x 8 heads per n-tile)
+    float sacc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+    {
+      const int r = lane & 15;  // key row of this lane's ldmatrix address
+#pragma unroll
+      for (int ks = 0; ks < STEPS; ++ks) {
+        const int half = ks >> 2;
+        const int chunk = ((ks & 3) << 1) + (lane >> 4);  // 16-byte chunk within the half
+        uint32_t af[4];
+        ldsm_x4(kbase + half * kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), af);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
+      }
+    }
+
+    // ---- mask, online softmax (base 2), P in bf16
+    const int ts = sp.lo + t * KT;
+    const int row0 = tile_row0(t);
+    const bool valid0 = row0 + (lane >> 2) >= ts;      // key row lane/4
+    const bool valid1 = row0 + (lane >> 2) + 8 >= ts;  // key row lane/4 + 8
+    uint32_t plo[NT], phi[NT];
+    bool rescale = false;
+    float alpha[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float s0 = valid0 ? sacc[nt][0] * a.scale_log2 : -INFINITY;
+      const float s1 = valid0 ? sacc[nt][1] * a.scale_log2 : -INFINITY;
+      const float s2 = valid1 ? sacc[nt][2] * a.scale_log2 : -INFINITY;
+      const float s3 = valid1 ? sacc[nt][3] * a.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+      }
+      // every tile holds at least one valid key, so the new maxima are finite
+      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+      alpha[nt][0] = exp2f(m_run[nt][0] - mn0);
+      alpha[nt][1] = exp2f(m_run[nt][1] - mn1);
+      rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      plo[nt] = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
+      phi[nt] = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
+      l_run[nt][0] = fmaf(l_run[nt][0], alpha[nt][0], bf16lo_to_f32(plo[nt]) + bf16lo_to_f32(phi[nt]));
+      l_run[nt][1] = fmaf(l_run[nt][1], alpha[nt][1], bf16hi_to_f32(plo[nt]) + bf16hi_to_f32(phi[nt]));
+    }
+    if (__any_sync(kFull, rescale)) {
+#pragma unroll
+      for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          oacc[dt][nt][0] *= alpha[nt][0];
+          oacc[dt][nt][1] *= alpha[nt][1];
+          oacc[dt][nt][2] *= alpha[nt][0];
+          oacc[dt][nt][3] *= alpha[nt][1];
+        }
+    }
+
+    // ---- o^T += V^T P^T
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      pb[nt][0] = movmatrix_trans(plo[nt]);  // keys 0-7  -> B rows k 0-7
+      pb[nt][1] = movmatrix_trans(phi[nt]);  // keys 8-15 -> B rows k 8-15
+    }
+    {
+      const int key = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+      for (int dt = 0; dt < STEPS; ++dt) {
+        const int chunk = dt * 2 + ((lane >> 3) & 1);  // 16-byte chunk along d
+        const int half = chunk >> 3, cc = chunk & 7;
+        uint32_t af[4];
+        ldsm_x4_trans(vbase + half * kBoxBytes + key * 128 + ((cc ^ (key & 7)) << 4), af);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(oacc[dt][nt], af, pb[nt][0], pb[nt][1]);
+      }
+    }
+    __syncwarp();
+
+    // ---- refill this stage with the warp's tile NS steps ahead
+    const int tn = t + NS * NW;
+    if (lane == 0 && tn < ntiles) {
+      fence_proxy_async_smem();
+      issue(tn, s);
+    }
+  }
+
+  if (failed) {
+    // Record the error, then let every load this warp issued land (bounded)
+    // before the CTA reuses or releases its shared memory.
+    if (lane == 0) raise_status(kStatusTimeout);
+    const int my_tiles = (ntiles > warp) ? (ntiles - warp + NW - 1) / NW : 0;
+    const int last = min(it + NS, my_tiles);
+    for (int i = it; i < last; ++i) mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+      for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[dt][nt][e] = 0.f;
+    }
+  }
+
+  // denominators: sum over the 8 lanes that share a head column
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) l_run[nt][j] += __shfl_xor_sync(kFull, l_run[nt][j], o);
+
+  __syncthreads();  // every warp is done with its stages: reuse them for o
+  float* sm_o = reinterpret_cast<float*>(stages);
+  if (lane < 4) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        sm_m[warp * HB + nt * 8 + 2 * lane + j] = m_run[nt][j];
+        sm_l[warp * HB + nt * 8 + 2 * lane + j] = l_run[nt][j];
+      }
+  }
+#pragma unroll
+  for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
+        const int head = nt * 8 + 2 * (lane & 3) + (e & 1);
+        sm_o[(warp * HB + head) * D + d] = oacc[dt][nt][e];
+      }
+  __syncthreads();
+  emit_split_triplet<NW, HB, D>(sm_m, sm_l, sm_o, a, b, g, hb, slot);
+  if (MODE == kFused) fused_finish<NW, HB, D>(a, b, g, hb, sp.n_active, &sm_flag);
+}
+
+}  // namespace gqa

@@ -1,0 +1,448 @@
+// libgqadecode.so: the C ABI declared in include/gqa_decode.h.
+//
+// Host responsibilities only: argument checks, tensor-map encoding, the
+// workspace, and kernel launches on the caller's stream.  Every step of the
+// computation runs in the kernels of decode_tc.cuh (bf16), decode_simt.cuh
+// (fp32) and split_merge.cuh (merge).
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "gqa_decode.h"
+#include "decode_simt.cuh"
+#include "decode_tc.cuh"
+#include "split_merge.cuh"
+
+namespace {
+
+using namespace gqa;
+
+constexpr int kMaxSlots = 1024;
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
+
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+
+// ------------------------------------------------------------------ helpers
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Heads handled by one CTA for each path, and the number of head blocks.
+inline int tc_heads_per_cta(int G) { return G <= 8 ? 8 : 16; }
+inline int simt_heads_per_cta(int G) {
+  int hb = 1;
+  while (hb < G && hb < 16) hb <<= 1;
+  return hb;
+}
+inline int heads_per_cta(int dtype, int G) {
+  return dtype == GQA_BF16 ? tc_heads_per_cta(G) : simt_heads_per_cta(G);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view (d, kv head, row) of a packed bf16 cache; box = 64 d x 1 head x
+// 16 rows, 128-byte swizzle.  The row extent is a clip bound only: the
+// kernels never address a row at or past the batch's last row, and rows
+// below 0 (a shifted first tile) read zero fill.
+bool encode_cache_map(CUtensorMap* map, const void* base, int h_kv, int D) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(h_kv),
+                              static_cast<cuuint64_t>(1u) << 31};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                 static_cast<cuuint64_t>(h_kv) * D * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kTileKeys)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// One-time (per device) opt-in to large dynamic shared memory for a kernel.
+template <typename K>
+int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return GQA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return GQA_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return GQA_OK;
+}
+
+int after_launch() {
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------- kernel dispatch
+
+// Tensor-core kernel shape: NW warps per CTA, NS stages per warp.
+constexpr int kTcWarps = 4;
+constexpr int kTcStages = 4;
+
+template <int D, int NT, int MODE>
+int launch_tc(const DecodeArgs& a, const void* k, const void* v, dim3 grid, cudaStream_t st) {
+  constexpr int NW = kTcWarps, NS = kTcStages;
+  constexpr int smem = tc_dynamic_smem<D, NW, NS>();
+  static std::atomic<uint64_t> attr_done{0};
+  auto kern = decode_tc_bf16<D, NT, NW, NS, MODE>;
+  if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, k, a.h_kv, D) || !encode_cache_map(&vmap, v, a.h_kv, D))
+    return GQA_ERR_CUDA;
+  kern<<<grid, NW * 32, smem, st>>>(kmap, vmap, a);
+  return after_launch();
+}
+
+template <int D, int HB, int MODE>
+int launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
+  constexpr int NW = 4;
+  decode_simt_f32<D, HB, NW, MODE><<<grid, NW * 32, 0, st>>>(a);
+  return after_launch();
+}
+
+template <int D, int MODE>
+int launch_simt_hb(const DecodeArgs& a, int hb, dim3 grid, cudaStream_t st) {
+  switch (hb) {
+    case 1: return launch_simt<D, 1, MODE>(a, grid, st);
+    case 2: return launch_simt<D, 2, MODE>(a, grid, st);
+    case 4: return launch_simt<D, 4, MODE>(a, grid, st);
+    case 8: return launch_simt<D, 8, MODE>(a, grid, st);
+    default: return launch_simt<D, 16, MODE>(a, grid, st);
+  }
+}
+
+template <int MODE>
+int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
+  const int hb = heads_per_cta(dtype, a.G);
+  a.n_hb = (a.G + hb - 1) / hb;
+  const dim3 grid(a.n_slots, a.h_kv * a.n_hb, a.B);
+  if (dtype == GQA_BF16) {
+    const bool wide = hb == 16;
+    if (D == 128)
+      return wide ? launch_tc<128, 2, MODE>(a, a.k, a.v, grid, st)
+                  : launch_tc<128, 1, MODE>(a, a.k, a.v, grid, st);
+    return wide ? launch_tc<64, 2, MODE>(a, a.k, a.v, grid, st)
+                : launch_tc<64, 1, MODE>(a, a.k, a.v, grid, st);
+  }
+  if (D == 128) return launch_simt_hb<128, MODE>(a, hb, grid, st);
+  return launch_simt_hb<64, MODE>(a, hb, grid, st);
+}
+
+// ------------------------------------------------------------ validation
+
+struct Shape {
+  int B, h_q, h_kv, D, n_slots, n_splits, chunk_len, dtype;
+  float scale;
+};
+
+// Size / value checks that need no pointers.
+int check_shape(const Shape& s) {
+  if (s.B < 0 || s.h_q < 1 || s.h_kv < 1 || s.h_q % s.h_kv != 0) return GQA_ERR_INVALID_ARG;
+  if (s.dtype != GQA_F32 && s.dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (!std::isfinite(s.scale)) return GQA_ERR_INVALID_ARG;
+  if (s.D != 64 && s.D != 128) return s.D > 0 ? GQA_ERR_UNSUPPORTED : GQA_ERR_INVALID_ARG;
+  if (s.n_slots < 1 || s.n_slots > kMaxSlots) return GQA_ERR_INVALID_ARG;
+  if (s.B > 65535) return GQA_ERR_UNSUPPORTED;
+  const int G = s.h_q / s.h_kv;
+  const int hb = heads_per_cta(s.dtype, G);
+  if ((long long)s.h_kv * ((G + hb - 1) / hb) > 65535) return GQA_ERR_UNSUPPORTED;
+  return GQA_OK;
+}
+
+int check_common(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                 const Shape& s) {
+  if (int rc = check_shape(s)) return rc;
+  if (s.B == 0) return GQA_OK;
+  if (!q || !k || !v || !seqlens) return GQA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(seqlens, 4))
+    return GQA_ERR_INVALID_ARG;
+  return GQA_OK;
+}
+
+Shape split_shape(int B, int h_q, int h_kv, int D, int n_splits, float scale, int dtype) {
+  return Shape{B, h_q, h_kv, D, n_splits, n_splits, 0, dtype, scale};
+}
+
+Shape chunk_shape(int B, int h_q, int h_kv, int D, int chunk_len, int max_seqlen, float scale,
+                  int dtype) {
+  int slots = -1;
+  if (chunk_len >= 1 && max_seqlen >= 0) {
+    const long long n = ((long long)max_seqlen + chunk_len - 1) / chunk_len;
+    slots = n < 1 ? 1 : (n > kMaxSlots ? kMaxSlots + 1 : (int)n);
+  }
+  return Shape{B, h_q, h_kv, D, slots, 0, chunk_len, dtype, scale};
+}
+
+DecodeArgs make_args(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                     const Shape& s) {
+  DecodeArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.seqlens = seqlens;
+  a.B = s.B;
+  a.h_q = s.h_q;
+  a.h_kv = s.h_kv;
+  a.G = s.h_q / s.h_kv;
+  a.n_splits = s.n_splits;
+  a.chunk_len = s.chunk_len;
+  a.n_slots = s.n_slots;
+  a.scale_log2 = s.scale * kLog2e;
+  a.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  return a;
+}
+
+// ------------------------------------------------------------- workspace
+
+struct WsLayout {
+  size_t tickets, m, l, o, total;
+};
+
+// Both paths split a group into ceil(G / 16) head blocks when G > 16 and use
+// one block otherwise, so the layout does not depend on the dtype.
+WsLayout ws_layout(const Shape& s) {
+  const int G = s.h_q / s.h_kv;
+  const size_t n_tickets = (size_t)s.B * s.h_kv * (G <= 16 ? 1 : (G + 15) / 16);
+  const size_t rows = (size_t)s.B * s.h_q;
+  WsLayout w;
+  w.tickets = 0;
+  w.m = round_up(n_tickets * sizeof(int), 256);
+  w.l = w.m + round_up(rows * s.n_slots * sizeof(float), 256);
+  w.o = w.l + round_up(rows * s.n_slots * sizeof(float), 256);
+  w.total = w.o + round_up(rows * s.n_slots * s.D * sizeof(float), 256);
+  return w;
+}
+
+struct LibWorkspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+LibWorkspace g_ws[kMaxDevices];
+
+// Library-owned, zero-filled, grow-only workspace of the current device.
+int lib_workspace(size_t need, void** out) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  LibWorkspace& w = g_ws[dev];
+  if (w.bytes < need) {
+    if (w.ptr) {
+      if (cudaDeviceSynchronize() != cudaSuccess) return GQA_ERR_CUDA;
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    const size_t bytes = round_up(need, 1 << 20);
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return GQA_ERR_WORKSPACE;
+    if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaFree(p);
+      return GQA_ERR_CUDA;
+    }
+    w.ptr = p;
+    w.bytes = bytes;
+  }
+  *out = w.ptr;
+  return GQA_OK;
+}
+
+int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, float* out,
+          const Shape& s, void* workspace, size_t workspace_bytes, void* stream) {
+  if (int rc = check_common(q, k, v, seqlens, s)) return rc;
+  if (s.B == 0) return GQA_OK;
+  if (!out || !aligned(out, 16)) return GQA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(s);
+  void* ws = workspace;
+  if (ws) {
+    if (workspace_bytes < w.total || !aligned(ws, 256)) return GQA_ERR_WORKSPACE;
+  } else if (int rc = lib_workspace(w.total, &ws)) {
+    return rc;
+  }
+  DecodeArgs a = make_args(q, k, v, seqlens, s);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  a.tickets = reinterpret_cast<int*>(base + w.tickets);
+  a.m = reinterpret_cast<float*>(base + w.m);
+  a.l = reinterpret_cast<float*>(base + w.l);
+  a.o = reinterpret_cast<float*>(base + w.o);
+  a.out = out;
+  return launch_decode<kFused>(a, s.dtype, s.D, as_stream(stream));
+}
+
+int partial(const void* q, const void* k, const void* v, const int32_t* seqlens, float* m,
+            float* l, float* o, const Shape& s, void* stream) {
+  if (int rc = check_common(q, k, v, seqlens, s)) return rc;
+  if (s.B == 0) return GQA_OK;
+  if (!m || !l || !o || !aligned(m, 16) || !aligned(l, 16) || !aligned(o, 16))
+    return GQA_ERR_INVALID_ARG;
+  DecodeArgs a = make_args(q, k, v, seqlens, s);
+  a.m = m;
+  a.l = l;
+  a.o = o;
+  return launch_decode<kPartial>(a, s.dtype, s.D, as_stream(stream));
+}
+
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // No thread ever arrives on `bar`: the wait must run out and report it.
+  if (threadIdx.x == 0 && !mbar_wait_bounded(smem_u32(&bar), 0, timeout_ns))
+    raise_status(kStatusTimeout);
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" {
+
+int gqa_decode_version(void) { return 100; }
+
+const char* gqa_decode_error_string(int status) {
+  switch (status) {
+    case GQA_OK: return "GQA_OK";
+    case GQA_ERR_INVALID_ARG: return "GQA_ERR_INVALID_ARG: invalid argument";
+    case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED: valid but unsupported shape";
+    case GQA_ERR_CUDA: return "GQA_ERR_CUDA: a CUDA call failed";
+    case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE: workspace too small, misaligned or not allocatable";
+    case GQA_ERR_DEVICE_TIMEOUT: return "GQA_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
+    case GQA_ERR_DEVICE_SEQLEN: return "GQA_ERR_DEVICE_SEQLEN: a kernel saw S_b < 0 or S_b > max_seqlen";
+    default: return "unknown gqa_status";
+  }
+}
+
+size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits) {
+  const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, 1.f, GQA_BF16);
+  return check_shape(s) ? 0 : ws_layout(s).total;
+}
+
+size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head, int chunk_len,
+                                         int max_seqlen) {
+  const Shape s = chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, 1.f, GQA_BF16);
+  return check_shape(s) ? 0 : ws_layout(s).total;
+}
+
+int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* seqlens, float* out, int B, int h_q, int h_kv, int d_head,
+                    int n_splits, float scale, int dtype, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return fused(q, k_cache, v_cache, seqlens, out,
+               split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype), workspace,
+               workspace_bytes, stream);
+}
+
+int gqa_decode_attn_chunked(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* seqlens, float* out, int B, int h_q, int h_kv,
+                            int d_head, int chunk_len, int max_seqlen, float scale, int dtype,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return fused(q, k_cache, v_cache, seqlens, out,
+               chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, scale, dtype), workspace,
+               workspace_bytes, stream);
+}
+
+int gqa_decode_partial(const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* seqlens, float* m, float* l, float* o, int B, int h_q,
+                       int h_kv, int d_head, int n_splits, float scale, int dtype, void* stream) {
+  return partial(q, k_cache, v_cache, seqlens, m, l, o,
+                 split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype), stream);
+}
+
+int gqa_decode_partial_chunked(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* seqlens, float* m, float* l, float* o, int B,
+                               int h_q, int h_kv, int d_head, int chunk_len, int max_seqlen,
+                               float scale, int dtype, void* stream) {
+  return partial(q, k_cache, v_cache, seqlens, m, l, o,
+                 chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, scale, dtype), stream);
+}
+
+int mlo_merge(const float* m, const float* l, const float* o, float* out, int rows, int n_splits,
+              int d_head, void* stream) {
+  if (rows < 0 || n_splits < 1 || d_head < 1 || d_head > 256) return GQA_ERR_INVALID_ARG;
+  if (rows == 0) return GQA_OK;
+  if (!m || !l || !o || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned(m, 4) || !aligned(l, 4) || !aligned(o, 4) || !aligned(out, 4))
+    return GQA_ERR_INVALID_ARG;
+  const dim3 grid((rows + 3) / 4);
+  cudaStream_t st = as_stream(stream);
+  if (d_head <= 64)
+    mlo_merge_kernel<2><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
+  else if (d_head <= 128)
+    mlo_merge_kernel<4><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
+  else
+    mlo_merge_kernel<8><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
+  return after_launch();
+}
+
+int gqa_decode_get_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return GQA_ERR_CUDA;
+  if (word) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return GQA_ERR_CUDA;
+  }
+  if (word & kStatusTimeout) return GQA_ERR_DEVICE_TIMEOUT;
+  if (word & (kStatusNegSeqlen | kStatusSeqlenOverMax)) return GQA_ERR_DEVICE_SEQLEN;
+  return GQA_OK;
+}
+
+int gqa_decode_set_wait_timeout_ns(unsigned long long timeout_ns) {
+  g_timeout_ns.store(timeout_ns ? timeout_ns : kDefaultTimeoutNs, std::memory_order_relaxed);
+  return GQA_OK;
+}
+
+int gqa_decode_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns == 0 || timeout_ns > 10ull * kDefaultTimeoutNs) return GQA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
+  return after_launch();
+}
+
+int gqa_decode_release(void) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  LibWorkspace& w = g_ws[dev];
+  if (w.ptr) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return GQA_ERR_CUDA;
+    cudaFree(w.ptr);
+    w.ptr = nullptr;
+    w.bytes = 0;
+  }
+  return GQA_OK;
+}
+
+}  // extern "C"

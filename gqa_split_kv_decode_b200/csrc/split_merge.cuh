@@ -1,0 +1,221 @@
+// Split assignment, triplet emission and the log-sum-exp merge shared by the
+// decode kernels and mlo_merge.
+//
+// Method (kernbench "_attention_mesh_mlo.py", attention_mesh_mlo_kernel): each
+// shard of the sequence yields a triplet (m, l, o) -- the maximum logit, the
+// softmax denominator relative to it and the unnormalised weighted sum of V
+// ("One-shot local partial attention"); triplets combine with
+// m_c = max(m, m'), l = l e^{m-m_c} + l' e^{m'-m_c}, o = o e^{m-m_c} +
+// o' e^{m'-m_c}, and the answer is o / l ("Final normalize").  Merging all n
+// triplets against their common maximum M is the same rule applied n - 1
+// times, written in one pass.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace gqa {
+
+// Everything a decode kernel needs besides the tensor maps.
+struct DecodeArgs {
+  const void* q;            // [B][h_q][D]
+  const void* k;            // packed [rows][h_kv][D] (SIMT path reads it directly)
+  const void* v;
+  const int32_t* seqlens;   // [B]
+  float* m;                 // triplets: m, l [B*h_q][n_slots], o [B*h_q][n_slots][D]
+  float* l;
+  float* o;
+  float* out;               // fused: [B*h_q][D]
+  int* tickets;             // fused: one counter per (b, blockIdx.y)
+  int B, h_q, h_kv, G, n_hb;
+  int n_splits;             // > 0: split by count
+  int chunk_len;            // > 0: split by fixed chunks
+  int n_slots;              // triplet slots per row == gridDim.x
+  float scale_log2;         // scale * log2(e): logits are kept in base 2
+  unsigned long long timeout_ns;
+};
+
+enum { kPartial = 0, kFused = 1 };
+
+struct Split {
+  long long off;  // packed row of the sequence's first key
+  int S;          // sequence length (negative lengths read as 0)
+  int lo, hi;     // this split's keys [lo, hi), relative to the sequence
+  int n_active;   // splits of this sequence that hold keys (>= 1)
+};
+
+// Sequence b's packed offset and the key range of split `slot` (whole warp).
+// Split i covers [i*L, min((i+1)*L, S)) with L = ceil(S / n_splits) or
+// L = chunk_len.  n_active = max(1, ceil(S / L)): the number of splits the
+// fused merge waits for (split 0 stands in for an empty sequence).
+__device__ __forceinline__ Split locate_split(const DecodeArgs& a, int b, int slot, int lane,
+                                              bool report) {
+  long long acc = 0;
+  for (int j = lane; j < b; j += 32) {
+    const int s = __ldg(a.seqlens + j);
+    acc += s > 0 ? s : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+  int S = __ldg(a.seqlens + b);
+  if (S < 0) {
+    if (report) raise_status(kStatusNegSeqlen);
+    S = 0;
+  }
+  const long long L =
+      a.n_splits > 0 ? ((long long)S + a.n_splits - 1) / a.n_splits : (long long)a.chunk_len;
+  int n_active = S > 0 ? (int)(((long long)S + L - 1) / L) : 1;
+  if (n_active > a.n_slots) {
+    if (report) raise_status(kStatusSeqlenOverMax);
+    n_active = a.n_slots;
+  }
+  long long lo = (long long)slot * L;
+  if (lo > S) lo = S;
+  long long hi = lo + L;
+  if (hi > S) hi = S;
+  Split sp;
+  sp.off = acc;
+  sp.S = S;
+  sp.lo = (int)lo;
+  sp.hi = (int)hi;
+  sp.n_active = n_active;
+  return sp;
+}
+
+__device__ __forceinline__ size_t query_row(const DecodeArgs& a, int b, int g, int gi) {
+  return (size_t)b * a.h_q + (size_t)g * a.G + gi;
+}
+
+// Writes the empty triplet (-inf, 0, 0) of split `slot` for the CTA's heads.
+template <int HB, int D>
+__device__ void emit_empty_triplet(const DecodeArgs& a, int b, int g, int hb, int slot) {
+  for (int idx = threadIdx.x; idx < HB * D; idx += blockDim.x) {
+    const int hh = idx / D, dd = idx % D;
+    const int gi = hb * HB + hh;
+    if (gi >= a.G) continue;
+    const size_t row = query_row(a, b, g, gi);
+    a.o[(row * a.n_slots + slot) * D + dd] = 0.f;
+    if (dd == 0) {
+      a.m[row * a.n_slots + slot] = -INFINITY;
+      a.l[row * a.n_slots + slot] = 0.f;
+    }
+  }
+}
+
+// Combines the NW per-warp triplets held in shared memory (m in base 2:
+// sm_m[w*HB+h]; sm_l likewise; sm_o[(w*HB+h)*D + d]) into this CTA's split
+// triplet and stores it at slot `slot` (m converted to natural-log units).
+template <int NW, int HB, int D>
+__device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const float* sm_o,
+                                   const DecodeArgs& a, int b, int g, int hb, int slot) {
+  for (int idx = threadIdx.x; idx < HB * D; idx += blockDim.x) {
+    const int hh = idx / D, dd = idx % D;
+    const int gi = hb * HB + hh;
+    if (gi >= a.G) continue;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w * HB + hh]);
+    float ov = 0.f, lv = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float sc = exp2f(sm_m[w * HB + hh] - M);
+        ov = fmaf(sm_o[(w * HB + hh) * D + dd], sc, ov);
+        lv = fmaf(sm_l[w * HB + hh], sc, lv);
+      }
+    }
+    const size_t row = query_row(a, b, g, gi);
+    a.o[(row * a.n_slots + slot) * D + dd] = ov;
+    if (dd == 0) {
+      a.m[row * a.n_slots + slot] = (M == -INFINITY) ? -INFINITY : M * kLn2;
+      a.l[row * a.n_slots + slot] = lv;
+    }
+  }
+}
+
+// Merges n triplets of one row and normalises: the whole warp cooperates,
+// lane j owning elements j, j+32, ... (d <= 32*MAXK).  Splits are combined
+// strictly in index order, so every element's result is deterministic and
+// identical wherever this function runs.  m in natural-log units.
+template <int MAXK>
+__device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
+                                               int n, int d, float* out, int lane) {
+  float M = -INFINITY;
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(m + i));
+  M = warp_max(M);
+  float acc[MAXK];
+#pragma unroll
+  for (int k = 0; k < MAXK; ++k) acc[k] = 0.f;
+  float L = 0.f;
+  if (M != -INFINITY) {
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      float wi = 0.f, li = 0.f;
+      if (i < n) {
+        wi = exp2f((__ldcg(m + i) - M) * kLog2e);  // 0 for an empty split
+        li = __ldcg(l + i);
+      }
+      const int cnt = min(32, n - base);
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(kFull, wi, j);
+        const float lj = __shfl_sync(kFull, li, j);
+        L = fmaf(lj, wj, L);
+        const float* oj = o + (size_t)(base + j) * d;
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) {
+          const int dd = lane + 32 * k;
+          if (dd < d) acc[k] = fmaf(__ldcg(oj + dd), wj, acc[k]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < MAXK; ++k) {
+    const int dd = lane + 32 * k;
+    if (dd < d) out[dd] = L > 0.f ? acc[k] / L : 0.f;
+  }
+}
+
+// Fused finish: after this CTA's triplet is stored, take a ticket for the
+// (b, kv head, head block); the CTA that takes the last one merges the
+// group's rows over the n_active splits and writes `out`.  Nothing waits on
+// another CTA, so there is no inter-CTA spin.  The last CTA also resets the
+// ticket to 0 for the next call.
+template <int NW, int HB, int D>
+__device__ void fused_finish(const DecodeArgs& a, int b, int g, int hb, int n_active,
+                             int* sm_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* t = a.tickets + (size_t)b * gridDim.y + blockIdx.y;
+    const int prev = atomicAdd(t, 1);
+    const int last = (prev == n_active - 1);
+    if (last) atomicExch(t, 0);
+    *sm_flag = last;
+  }
+  __syncthreads();
+  if (!*sm_flag) return;
+  __threadfence();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int hh = warp; hh < HB; hh += NW) {
+    const int gi = hb * HB + hh;
+    if (gi >= a.G) break;
+    const size_t row = query_row(a, b, g, gi);
+    merge_row_warp<D / 32>(a.m + row * a.n_slots, a.l + row * a.n_slots,
+                           a.o + row * a.n_slots * D, n_active, D, a.out + row * D, lane);
+  }
+}
+
+// Stand-alone merge: one warp per row.
+template <int MAXK>
+__global__ void __launch_bounds__(128) mlo_merge_kernel(const float* __restrict__ m,
+                                                        const float* __restrict__ l,
+                                                        const float* __restrict__ o,
+                                                        float* __restrict__ out, int rows, int n,
+                                                        int d) {
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  merge_row_warp<MAXK>(m + (size_t)row * n, l + (size_t)row * n, o + (size_t)row * n * d, n, d,
+                       out + (size_t)row * d, threadIdx.x & 31);
+}
+
+}  // namespace gqa

@@ -1,0 +1,191 @@
+/*
+ * gqa_decode.h -- C ABI of libgqadecode.so: grouped-query decode attention
+ * over a sequence-split KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method (kernbench "_attention_mesh_mlo.py", decode kernel
+ * attention_mesh_mlo_kernel and its module docstring): the single-token query
+ * Q is replicated, the KV cache is cut along the sequence into contiguous
+ * shards; each shard computes its partial attention as a triplet
+ *     m = max_j s_j,   l = sum_j exp(s_j - m),   o = sum_j exp(s_j - m) v_j
+ * ("One-shot local partial attention"), the triplets are combined with the
+ * log-sum-exp rule (m_c = max(m, m'), l = l e^{m-m_c} + l' e^{m'-m_c},
+ * o = o e^{m-m_c} + o' e^{m'-m_c}) and the result is O = o / l ("Final
+ * normalize").  Here the shards are split-KV chunks on one GPU.
+ *
+ * Logits: s_j = scale * <q[b][h][:], k[row][g][:]> where query head h reads
+ * kv head g = floor(h / (h_q / h_kv)) (contiguous groups, as in the tinygrad
+ * "llama speed tracking" page's Attention.__call__, which shards q by
+ * n_rep * head_dim beside k and v by head_dim).
+ *
+ * ---------------------------------------------------------------- layouts
+ *   q        [B][h_q][d_head]            dtype (fp32 or bf16), contiguous
+ *   k_cache  [sum_b S_b][h_kv][d_head]   dtype, packed: sequence b occupies
+ *   v_cache  [sum_b S_b][h_kv][d_head]   rows S_0 + ... + S_{b-1} onwards
+ *   seqlens  int32 [B]                   S_b (device memory)
+ *   out      fp32 [B][h_q][d_head]       O = o / l (0 where S_b == 0)
+ *   m, l     fp32 [B][h_q][n_slots]      per-split triplets (m in natural
+ *   o        fp32 [B][h_q][n_slots][d_head]   log units, o unnormalised)
+ * With every S_b equal to S the packed cache is the dense [B][S][h_kv][d]
+ * layout.
+ *
+ * Split policies (the page splits evenly, 1/n_ranks per rank):
+ *   by count: split i of sequence b covers [i*L_b, min((i+1)*L_b, S_b)),
+ *             L_b = ceil(S_b / n_splits); n_slots = n_splits;
+ *   chunked:  split i covers [i*chunk_len, min((i+1)*chunk_len, S_b)),
+ *             n_slots = max(1, ceil(max_seqlen / chunk_len)).
+ * An empty split's triplet is (-inf, 0, 0).
+ *
+ * ------------------------------------------------------------ conventions
+ * - Every pointer argument is a DEVICE pointer on the current CUDA device and
+ *   is owned by the caller, except `workspace == NULL` (see below).
+ * - q, k_cache, v_cache and every fp32 output must be 16-byte aligned.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call is asynchronous on that stream and never
+ *   synchronises the host, except for workspace growth (below) and
+ *   gqa_decode_get_status().
+ * - Arguments are checked on the host; on any error the call returns a
+ *   nonzero gqa_status and launches nothing.  Supported: d_head in {64, 128};
+ *   h_q % h_kv == 0; 1 <= n_splits <= 1024 (n_slots <= 1024 when chunked);
+ *   finite scale; dtype GQA_F32 or GQA_BF16 (q, k and v share it).
+ * - Errors that only the device can see (a negative S_b, S_b above
+ *   max_seqlen in chunked mode, a bounded wait that ran out) set bits of a
+ *   per-device status word, read and cleared by gqa_decode_get_status().
+ * - No stray reads: a kernel reads only cache rows that belong to the batch
+ *   (rows [0, sum_b S_b)); rows of a neighbouring sequence that fall inside a
+ *   loaded tile are masked by index, so they must hold finite values (any
+ *   packed cache does).
+ */
+#ifndef GQA_DECODE_H
+#define GQA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or value */
+    GQA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. d_head 96) */
+    GQA_ERR_CUDA = 3,            /* a CUDA runtime / driver call failed */
+    GQA_ERR_WORKSPACE = 4,       /* caller workspace too small or misaligned */
+    GQA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait in a kernel ran out */
+    GQA_ERR_DEVICE_SEQLEN = 6    /* a kernel saw S_b < 0 or S_b > max_seqlen */
+} gqa_status;
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+GQA_API int gqa_decode_version(void);
+
+/* Human-readable name of a gqa_status value (static storage). */
+GQA_API const char *gqa_decode_error_string(int status);
+
+/* Bytes of workspace gqa_decode_attn needs: one ticket counter per
+ * (b, kv head, head block) plus fp32 triplets for every (b, h, split).
+ * Returns 0 for arguments gqa_decode_attn would reject. */
+GQA_API size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits);
+
+/* Same for gqa_decode_attn_chunked. */
+GQA_API size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head,
+                                         int chunk_len, int max_seqlen);
+
+/*
+ * Fused decode attention, split by count: one kernel computes every split's
+ * triplet and the last split to finish for a (b, kv head) merges them in
+ * split order and writes out[b][h][:] for the group's query heads.  The
+ * result is identical to gqa_decode_partial followed by mlo_merge.
+ *
+ * workspace: NULL, or caller device memory of at least
+ *   gqa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED
+ *   before its first use.  Every call that completes leaves its ticket
+ *   counters at zero again, so a workspace is reusable without clearing;
+ *   after a device error (status word set) zero it again.  Calls that share a
+ *   workspace must be ordered on one stream.  With NULL the library uses a
+ *   grow-only workspace of its own per device (growing it synchronises the
+ *   device); calls that use it must be ordered on one stream.
+ */
+GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *seqlens, float *out,
+                    int B, int h_q, int h_kv, int d_head, int n_splits, float scale,
+                    int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Fused decode attention with fixed-length chunks (ragged batches): split i
+ * of sequence b covers [i*chunk_len, min((i+1)*chunk_len, S_b)); the last
+ * chunk may be partial.  max_seqlen bounds every S_b (host-known, so no
+ * device-to-host copy is needed); a larger S_b sets GQA_ERR_DEVICE_SEQLEN in
+ * the status word and only its first n_slots chunks are used.
+ */
+GQA_API int gqa_decode_attn_chunked(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, float *out,
+                            int B, int h_q, int h_kv, int d_head, int chunk_len, int max_seqlen,
+                            float scale, int dtype, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/*
+ * Partial attention only ("One-shot local partial attention" of the page, one
+ * split per shard): writes the (m, l, o) triplet of every (b, h, split) into
+ * m, l [B][h_q][n_splits] and o [B][h_q][n_splits][d_head] (fp32, m in
+ * natural-log units, o unnormalised, empty split = (-inf, 0, 0)).
+ */
+GQA_API int gqa_decode_partial(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *seqlens, float *m, float *l, float *o,
+                       int B, int h_q, int h_kv, int d_head, int n_splits, float scale,
+                       int dtype, void *stream);
+
+/* Partial attention with the chunked split policy (n_slots triplets per row,
+ * n_slots = max(1, ceil(max_seqlen / chunk_len))). */
+GQA_API int gqa_decode_partial_chunked(const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *seqlens, float *m, float *l, float *o,
+                               int B, int h_q, int h_kv, int d_head, int chunk_len,
+                               int max_seqlen, float scale, int dtype, void *stream);
+
+/*
+ * Log-sum-exp merge and normalisation of n_splits triplets per row (the
+ * page's merge of received triplets, then "Final normalize"):
+ *   M = max_i m_i,  l* = sum_i l_i e^{m_i - M},  o* = sum_i o_i e^{m_i - M},
+ *   out = o* / l*   (0 when every triplet of the row is empty).
+ * m, l: fp32 [rows][n_splits]; o: fp32 [rows][n_splits][d_head];
+ * out: fp32 [rows][d_head].  Splits are summed in index order, so the result
+ * is deterministic.  1 <= d_head <= 256, n_splits >= 1.
+ */
+GQA_API int mlo_merge(const float *m, const float *l, const float *o, float *out,
+              int rows, int n_splits, int d_head, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's status word.
+ * Returns GQA_OK, GQA_ERR_DEVICE_TIMEOUT, GQA_ERR_DEVICE_SEQLEN or
+ * GQA_ERR_CUDA.
+ */
+GQA_API int gqa_decode_get_status(void *stream);
+
+/* Upper bound, in nanoseconds, on every wait inside the kernels (default
+ * 1e9).  A wait that runs out records GQA_ERR_DEVICE_TIMEOUT and the kernel
+ * returns without hanging.  0 restores the default. */
+GQA_API int gqa_decode_set_wait_timeout_ns(unsigned long long timeout_ns);
+
+/*
+ * Self-test of the bounded wait: launches one CTA that waits on a barrier no
+ * thread ever signals, with a bound of `timeout_ns`.  The wait runs out, the
+ * kernel records GQA_ERR_DEVICE_TIMEOUT in the status word and returns; the
+ * next gqa_decode_get_status() reports it.  Nothing else is touched.
+ */
+GQA_API int gqa_decode_selftest_wait_timeout(unsigned long long timeout_ns, void *stream);
+
+/* Frees this device's library-owned workspace (after synchronising it). */
+GQA_API int gqa_decode_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_DECODE_H */

@@ -1,0 +1,117 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host (no GPU needed: nothing here launches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gqa_split_kv_decode_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa_decode.h")
+
+OK, INVALID, UNSUPPORTED, CUDA_ERR, WORKSPACE = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = _build.build()
+    lib = ctypes.CDLL(path)
+    vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.gqa_decode_attn.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
+    lib.gqa_decode_attn_chunked.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
+    lib.gqa_decode_partial.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+    lib.mlo_merge.argtypes = [vp, vp, vp, vp, ci, ci, ci, vp]
+    lib.gqa_decode_workspace_size.restype = sz
+    lib.gqa_decode_workspace_size.argtypes = [ci] * 5
+    lib.gqa_decode_chunked_workspace_size.restype = sz
+    lib.gqa_decode_chunked_workspace_size.argtypes = [ci] * 6
+    lib.gqa_decode_error_string.restype = ctypes.c_char_p
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"GQA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_path():
+    names = set(declared_functions())
+    for required in ["gqa_decode_attn", "gqa_decode_partial", "mlo_merge", "gqa_decode_attn_chunked",
+                     "gqa_decode_get_status", "gqa_decode_workspace_size"]:
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in gqa_decode.h but not exported"
+
+
+def test_version_and_error_strings(lib):
+    assert lib.gqa_decode_version() >= 100
+    for code in range(7):
+        assert lib.gqa_decode_error_string(code).startswith(b"GQA_")
+    assert b"unknown" in lib.gqa_decode_error_string(99)
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(h_q=6, h_kv=4), INVALID),          # h_q not a multiple of h_kv
+    (dict(d=96), UNSUPPORTED),               # head dim other than 64 / 128
+    (dict(d=0), INVALID),
+    (dict(n_splits=0), INVALID),
+    (dict(n_splits=1025), INVALID),
+    (dict(scale=float("inf")), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(dtype=7), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(q=0), INVALID),                    # null pointer
+    (dict(k=FAKE + 8), INVALID),             # misaligned cache
+    (dict(out=FAKE + 4), INVALID),           # misaligned output
+    (dict(ws=FAKE, ws_bytes=16), WORKSPACE),  # caller workspace too small
+    (dict(ws=FAKE + 16, ws_bytes=1 << 30), WORKSPACE),  # not 256-byte aligned
+    (dict(B=0), OK),                         # empty batch: nothing to do
+])
+def test_fused_argument_checks(lib, kw, expect):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, out=FAKE, B=1, h_q=8, h_kv=2, d=128, n_splits=4,
+             scale=0.1, dtype=1, ws=None, ws_bytes=0)
+    a.update(kw)
+    rc = lib.gqa_decode_attn(a["q"], a["k"], a["v"], a["sl"], a["out"], a["B"], a["h_q"], a["h_kv"],
+                             a["d"], a["n_splits"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"], None)
+    assert rc == expect
+
+
+def test_chunked_argument_checks(lib):
+    args = [FAKE] * 5
+    assert lib.gqa_decode_attn_chunked(*args, 1, 8, 2, 128, 0, 100, 0.1, 1, None, 0, None) == INVALID
+    assert lib.gqa_decode_attn_chunked(*args, 1, 8, 2, 128, 16, -1, 0.1, 1, None, 0, None) == INVALID
+    # 1025 chunks of 1 key exceeds the 1024 triplet slots
+    assert lib.gqa_decode_attn_chunked(*args, 1, 8, 2, 128, 1, 1025, 0.1, 1, None, 0, None) == INVALID
+
+
+def test_partial_and_merge_argument_checks(lib):
+    p_null = [FAKE] * 4 + [0, FAKE, FAKE]
+    assert lib.gqa_decode_partial(*p_null, 1, 8, 2, 128, 4, 0.1, 1, None) == INVALID
+    assert lib.mlo_merge(FAKE, FAKE, FAKE, FAKE, 0, 4, 128, None) == OK     # no rows: no launch
+    assert lib.mlo_merge(FAKE, FAKE, FAKE, FAKE, 4, 0, 128, None) == INVALID
+    assert lib.mlo_merge(FAKE, FAKE, FAKE, FAKE, 4, 4, 257, None) == INVALID
+    assert lib.mlo_merge(0, FAKE, FAKE, FAKE, 4, 4, 128, None) == INVALID
+
+
+def test_workspace_size_arithmetic(lib):
+    # tickets (B * h_kv) + m + l (B*h_q*n fp32 each) + o (B*h_q*n*d fp32), 256-byte rounded
+    B, hq, hkv, d, n = 8, 64, 8, 128, 8
+    r = lambda x: (x + 255) // 256 * 256
+    expect = r(B * hkv * 4) + 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
+    assert lib.gqa_decode_workspace_size(B, hq, hkv, d, n) == expect
+    # groups above 16 heads use ceil(G / 16) head blocks, each with its own ticket
+    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == r(2 * 4) + 2 * r(32 * 2 * 4) + r(32 * 2 * 128 * 4)
+    assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == \
+        r(64 * 8 * 4) + 2 * r(64 * 32 * 32 * 4) + r(64 * 32 * 32 * 128 * 4)
+    assert lib.gqa_decode_workspace_size(1, 6, 4, 128, 4) == 0
+    assert lib.gqa_decode_workspace_size(1, 8, 2, 96, 4) == 0
