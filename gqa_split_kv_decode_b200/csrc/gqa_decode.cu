@@ -105,9 +105,16 @@ int after_launch() {
 
 // ---------------------------------------------------------- kernel dispatch
 
-// Tensor-core kernel shape: NW warps per CTA, NS stages per warp.
-constexpr int kTcWarps = 4;
-constexpr int kTcStages = 4;
+// Tensor-core kernel shape: NW warps per CTA, NS stages per warp (build-time
+// constants; -DGQA_TC_WARPS / -DGQA_TC_STAGES override them).
+#ifndef GQA_TC_WARPS
+#define GQA_TC_WARPS 4
+#endif
+#ifndef GQA_TC_STAGES
+#define GQA_TC_STAGES 4
+#endif
+constexpr int kTcWarps = GQA_TC_WARPS;
+constexpr int kTcStages = GQA_TC_STAGES;
 
 template <int D, int NT, int MODE>
 int launch_tc(const DecodeArgs& a, const void* k, const void* v, dim3 grid, cudaStream_t st) {
@@ -228,15 +235,24 @@ struct WsLayout {
   size_t tickets, m, l, o, total;
 };
 
-// Both paths split a group into ceil(G / 16) head blocks when G > 16 and use
-// one block otherwise, so the layout does not depend on the dtype.
-WsLayout ws_layout(const Shape& s) {
+// Workspace = a fixed 256 KiB ticket area, then the fp32 triplets.  The ticket
+// area has the same size and place for every shape, and each call returns the
+// tickets it used to zero, so the area is all zeros at rest whatever shapes
+// used the workspace before (triplets of one shape never land on tickets of
+// another).  Both paths split a group into ceil(G / 16) head blocks when
+// G > 16 and use one block otherwise, so the layout does not depend on dtype.
+constexpr size_t kTicketBytes = 256 * 1024;
+
+size_t n_tickets(const Shape& s) {
   const int G = s.h_q / s.h_kv;
-  const size_t n_tickets = (size_t)s.B * s.h_kv * (G <= 16 ? 1 : (G + 15) / 16);
+  return (size_t)s.B * s.h_kv * (G <= 16 ? 1 : (G + 15) / 16);
+}
+
+WsLayout ws_layout(const Shape& s) {
   const size_t rows = (size_t)s.B * s.h_q;
   WsLayout w;
   w.tickets = 0;
-  w.m = round_up(n_tickets * sizeof(int), 256);
+  w.m = kTicketBytes;
   w.l = w.m + round_up(rows * s.n_slots * sizeof(float), 256);
   w.o = w.l + round_up(rows * s.n_slots * sizeof(float), 256);
   w.total = w.o + round_up(rows * s.n_slots * s.D * sizeof(float), 256);
@@ -280,6 +296,7 @@ int lib_workspace(size_t need, void** out) {
 int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, float* out,
           const Shape& s, void* workspace, size_t workspace_bytes, void* stream) {
   if (int rc = check_common(q, k, v, seqlens, s)) return rc;
+  if (n_tickets(s) * sizeof(int) > kTicketBytes) return GQA_ERR_UNSUPPORTED;
   if (s.B == 0) return GQA_OK;
   if (!out || !aligned(out, 16)) return GQA_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(s);
@@ -347,13 +364,15 @@ const char* gqa_decode_error_string(int status) {
 
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits) {
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, 1.f, GQA_BF16);
-  return check_shape(s) ? 0 : ws_layout(s).total;
+  if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
+  return ws_layout(s).total;
 }
 
 size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head, int chunk_len,
                                          int max_seqlen) {
   const Shape s = chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, 1.f, GQA_BF16);
-  return check_shape(s) ? 0 : ws_layout(s).total;
+  if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
+  return ws_layout(s).total;
 }
 
 int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,

@@ -89,9 +89,10 @@ GQA_API int gqa_decode_version(void);
 /* Human-readable name of a gqa_status value (static storage). */
 GQA_API const char *gqa_decode_error_string(int status);
 
-/* Bytes of workspace gqa_decode_attn needs: one ticket counter per
- * (b, kv head, head block) plus fp32 triplets for every (b, h, split).
- * Returns 0 for arguments gqa_decode_attn would reject. */
+/* Bytes of workspace gqa_decode_attn needs: a fixed 256 KiB ticket area (one
+ * int32 counter per (b, kv head, head block); at most 65536 of them) followed
+ * by fp32 triplets for every (b, h, split).  Returns 0 for arguments
+ * gqa_decode_attn would reject. */
 GQA_API size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits);
 
 /* Same for gqa_decode_attn_chunked. */
@@ -105,11 +106,13 @@ GQA_API size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d
  * result is identical to gqa_decode_partial followed by mlo_merge.
  *
  * workspace: NULL, or caller device memory of at least
- *   gqa_decode_workspace_size(...) bytes, 256-byte aligned, ZERO-FILLED
- *   before its first use.  Every call that completes leaves its ticket
- *   counters at zero again, so a workspace is reusable without clearing;
- *   after a device error (status word set) zero it again.  Calls that share a
- *   workspace must be ordered on one stream.  With NULL the library uses a
+ *   gqa_decode_workspace_size(...) bytes, 256-byte aligned, whose first
+ *   256 KiB (the ticket area) are ZERO-FILLED before its first use.  Every
+ *   call that completes returns the tickets it used to zero and writes
+ *   triplets only past the ticket area, so one workspace serves calls of any
+ *   shape without clearing; after a device error (status word set) zero the
+ *   ticket area again.  Calls that share a workspace must be ordered on one
+ *   stream.  With NULL the library uses a
  *   grow-only workspace of its own per device (growing it synchronises the
  *   device); calls that use it must be ordered on one stream.
  */

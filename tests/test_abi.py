@@ -104,14 +104,16 @@ def test_partial_and_merge_argument_checks(lib):
 
 
 def test_workspace_size_arithmetic(lib):
-    # tickets (B * h_kv) + m + l (B*h_q*n fp32 each) + o (B*h_q*n*d fp32), 256-byte rounded
+    # fixed 256 KiB ticket area + m + l (B*h_q*n fp32 each) + o (B*h_q*n*d fp32), 256-byte rounded
     B, hq, hkv, d, n = 8, 64, 8, 128, 8
     r = lambda x: (x + 255) // 256 * 256
-    expect = r(B * hkv * 4) + 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
+    T = 256 * 1024
+    expect = T + 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
     assert lib.gqa_decode_workspace_size(B, hq, hkv, d, n) == expect
-    # groups above 16 heads use ceil(G / 16) head blocks, each with its own ticket
-    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == r(2 * 4) + 2 * r(32 * 2 * 4) + r(32 * 2 * 128 * 4)
+    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == T + 2 * r(32 * 2 * 4) + r(32 * 2 * 128 * 4)
     assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == \
-        r(64 * 8 * 4) + 2 * r(64 * 32 * 32 * 4) + r(64 * 32 * 32 * 128 * 4)
+        T + 2 * r(64 * 32 * 32 * 4) + r(64 * 32 * 32 * 128 * 4)
+    # more than 65536 tickets (B * h_kv * head blocks) is refused
+    assert lib.gqa_decode_workspace_size(65535, 8, 2, 128, 1) == 0
     assert lib.gqa_decode_workspace_size(1, 6, 4, 128, 4) == 0
     assert lib.gqa_decode_workspace_size(1, 8, 2, 96, 4) == 0
