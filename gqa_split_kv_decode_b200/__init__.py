@@ -110,6 +110,21 @@ def _inputs(q, k_cache, v_cache, seqlens):
     return B, h_q, k_cache.shape[1], d, _dtype_code(q)
 
 
+_dummies: dict = {}
+
+
+def _ptr(t: torch.Tensor) -> int:
+    """Device address of a tensor; an empty tensor (a cache with no rows)
+    gets a small zeroed placeholder, which the kernels never read because
+    every sequence of such a batch has length 0."""
+    if t.numel() > 0:
+        return t.data_ptr()
+    key = (t.device.type, t.device.index)
+    if key not in _dummies:
+        _dummies[key] = torch.zeros(256, dtype=torch.uint8, device=t.device)
+    return _dummies[key].data_ptr()
+
+
 def _default_scale(d: int, scale):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
@@ -154,7 +169,7 @@ def gqa_decode_attn(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, out
     if workspace is None:
         workspace = _workspace(q.device, need)
     with torch.cuda.device(q.device):
-        _check(_attn(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+        _check(_attn(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
                      out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                      _stream(q.device)), "gqa_decode_attn")
@@ -170,7 +185,7 @@ def gqa_decode_attn_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_se
     if workspace is None:
         workspace = _workspace(q.device, need)
     with torch.cuda.device(q.device):
-        _check(_attn_chunked(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+        _check(_attn_chunked(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
                              out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
                              _default_scale(d, scale), dt, workspace.data_ptr(),
                              workspace.numel() * workspace.element_size(), _stream(q.device)),
@@ -190,7 +205,7 @@ def gqa_decode_partial(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, 
     B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
     m, l, o = _triplets(B, h_q, n_splits, d, q.device, m, l, o)
     with torch.cuda.device(q.device):
-        _check(_partial(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(),
+        _check(_partial(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
                         m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
                         _default_scale(d, scale), dt, _stream(q.device)), "gqa_decode_partial")
     return m, l, o
@@ -203,7 +218,7 @@ def gqa_decode_partial_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max
     n = max(1, -(-max_seqlen // chunk_len)) if chunk_len > 0 and max_seqlen >= 0 else 1
     m, l, o = _triplets(B, h_q, n, d, q.device, m, l, o)
     with torch.cuda.device(q.device):
-        _check(_partial_chunked(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        _check(_partial_chunked(q.data_ptr(), _ptr(k_cache), _ptr(v_cache),
                                 seqlens.data_ptr(), m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q,
                                 h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
                                 _stream(q.device)), "gqa_decode_partial_chunked")

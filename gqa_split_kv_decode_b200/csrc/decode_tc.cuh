@@ -18,8 +18,8 @@
 // the whole split; the S^T accumulator becomes P^T's B fragment through one
 // movmatrix transpose per 8x8 block.  Softmax statistics are fp32 in base 2
 // (scale * log2 e is folded into one multiply), reduced with shuffles across
-// the 8 lanes that share a head.  P is rounded to bf16 for the PV product and
-// the denominator sums those same rounded weights.
+// the 8 lanes that share a head.  P enters the PV product as two bf16 parts
+// (hi + lo) so its rounding stays near fp32 level.
 //
 // The last tile of a split that is not a whole tile is loaded as the KT rows
 // that END at the split's end (shifted back) and the rows before the tile's
@@ -178,12 +178,12 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
 
-    // ---- mask, online softmax (base 2), P in bf16
+    // ---- mask, online softmax (base 2)
     const int ts = sp.lo + t * KT;
     const int row0 = tile_row0(t);
     const bool valid0 = row0 + (lane >> 2) >= ts;      // key row lane/4
     const bool valid1 = row0 + (lane >> 2) + 8 >= ts;  // key row lane/4 + 8
-    uint32_t plo[NT], phi[NT];
+    float p[NT][4];
     bool rescale = false;
     float alpha[NT][2];
 #pragma unroll
@@ -205,10 +205,12 @@ __global__ void __launch_bounds__(NW * 32)
       rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
       m_run[nt][0] = mn0;
       m_run[nt][1] = mn1;
-      plo[nt] = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
-      phi[nt] = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
-      l_run[nt][0] = fmaf(l_run[nt][0], alpha[nt][0], bf16lo_to_f32(plo[nt]) + bf16lo_to_f32(phi[nt]));
-      l_run[nt][1] = fmaf(l_run[nt][1], alpha[nt][1], bf16hi_to_f32(plo[nt]) + bf16hi_to_f32(phi[nt]));
+      p[nt][0] = exp2f(s0 - mn0);
+      p[nt][1] = exp2f(s1 - mn1);
+      p[nt][2] = exp2f(s2 - mn0);
+      p[nt][3] = exp2f(s3 - mn1);
+      l_run[nt][0] = fmaf(l_run[nt][0], alpha[nt][0], p[nt][0] + p[nt][2]);
+      l_run[nt][1] = fmaf(l_run[nt][1], alpha[nt][1], p[nt][1] + p[nt][3]);
     }
     if (__any_sync(kFull, rescale)) {
 #pragma unroll
@@ -222,12 +224,20 @@ __global__ void __launch_bounds__(NW * 32)
         }
     }
 
-    // ---- o^T += V^T P^T
-    uint32_t pb[NT][2];
+    // ---- o^T += V^T P^T.  P enters the bf16 product as hi + lo, two bf16
+    // parts whose sum carries ~16 significant bits, so a split of a few keys
+    // with large, opposite V rows keeps fp32-level accuracy.
+    uint32_t pb[NT][2][2];  // [n-tile][hi, lo][keys 0-7, keys 8-15]
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      pb[nt][0] = movmatrix_trans(plo[nt]);  // keys 0-7  -> B rows k 0-7
-      pb[nt][1] = movmatrix_trans(phi[nt]);  // keys 8-15 -> B rows k 8-15
+      const uint32_t h01 = pack_bf16x2(p[nt][0], p[nt][1]);
+      const uint32_t h23 = pack_bf16x2(p[nt][2], p[nt][3]);
+      const uint32_t l01 = pack_bf16x2(p[nt][0] - bf16lo_to_f32(h01), p[nt][1] - bf16hi_to_f32(h01));
+      const uint32_t l23 = pack_bf16x2(p[nt][2] - bf16lo_to_f32(h23), p[nt][3] - bf16hi_to_f32(h23));
+      pb[nt][0][0] = movmatrix_trans(h01);  // keys 0-7  -> B rows k 0-7
+      pb[nt][0][1] = movmatrix_trans(h23);  // keys 8-15 -> B rows k 8-15
+      pb[nt][1][0] = movmatrix_trans(l01);
+      pb[nt][1][1] = movmatrix_trans(l23);
     }
     {
       const int key = (lane & 7) + ((lane >> 4) << 3);
@@ -238,7 +248,10 @@ __global__ void __launch_bounds__(NW * 32)
         uint32_t af[4];
         ldsm_x4_trans(vbase + half * kBoxBytes + key * 128 + ((cc ^ (key & 7)) << 4), af);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(oacc[dt][nt], af, pb[nt][0], pb[nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_bf16_16816(oacc[dt][nt], af, pb[nt][0][0], pb[nt][0][1]);
+          mma_bf16_16816(oacc[dt][nt], af, pb[nt][1][0], pb[nt][1][1]);
+        }
       }
     }
     __syncwarp();

@@ -111,7 +111,7 @@ int after_launch() {
 #define GQA_TC_WARPS 4
 #endif
 #ifndef GQA_TC_STAGES
-#define GQA_TC_STAGES 4
+#define GQA_TC_STAGES 3
 #endif
 constexpr int kTcWarps = GQA_TC_WARPS;
 constexpr int kTcStages = GQA_TC_STAGES;
