@@ -1,6 +1,10 @@
 // bf16 decode attention: TMA-fed K/V tiles, tensor-core logits and PV.
 //
-// One CTA owns one (split, kv head g, head block, b).  Each of its NW warps
+// This file holds the per-tile math shared by both bf16 kernels and the
+// per-split kernel behind gqa_decode_partial; the fused kernel, which spreads
+// the same tiles evenly over persistent warps, is in decode_streamk.cuh.
+//
+// Per-split kernel: one CTA owns one (split, kv head g, head block, b).  Each of its NW warps
 // runs its own NS-stage TMA ring: a stage holds KT = 16 consecutive keys of K
 // and V for kv head g (one 64-element, 128-byte-swizzled box per half of
 // d_head), loaded once from HBM and shared by every query head of the group
@@ -46,7 +50,184 @@ constexpr int tc_dynamic_smem() {
   return NW * NS * TcShape<D>::kStageBytes + 1024;  // + slack for 1024-byte alignment
 }
 
-template <int D, int NT, int NW, int NS, int MODE>
+// Q^T as the B operand of S^T = K Q^T: thread holds head (lane / 4) of the
+// n-tile and d = 16 * ks + 2 * (lane % 4) + {0, 1} (b0) and + {8, 9} (b1).
+// Heads at or past G (padding of a partial block) read as zero.
+template <int D, int NT>
+__device__ __forceinline__ void load_q_frags(uint32_t (&qf)[NT][D / 16][2], const DecodeArgs& a,
+                                             int b, int g, int hb, int lane) {
+  constexpr int HB = NT * 8;
+  const uint32_t* qw = static_cast<const uint32_t*>(a.q);  // bf16 pairs
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int gi = hb * HB + nt * 8 + (lane >> 2);
+    const bool ok = gi < a.G;
+    const size_t base = (query_row(a, b, g, ok ? gi : 0) * D) / 2 + (lane & 3);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qf[nt][ks][0] = ok ? __ldg(qw + base + ks * 8) : 0u;
+      qf[nt][ks][1] = ok ? __ldg(qw + base + ks * 8 + 4) : 0u;
+    }
+  }
+}
+
+// Online-softmax state of one warp over the keys it has seen: per head
+// column (2 per lane and n-tile) the running max m (base 2) and this lane's
+// share of the denominator l; o^T accumulators in mma C-fragment layout
+// (d = 16 dt + lane/4 (+8), head = 8 nt + 2 (lane%4) (+1)).
+template <int D, int NT>
+struct WarpAcc {
+  float m[NT][2], l[NT][2];
+  float o[D / 16][NT][4];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[dt][nt][e] = 0.f;
+    }
+  }
+
+  // Sums each head's denominator over the 8 lanes that share its column.
+  __device__ __forceinline__ void reduce_l() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) l[nt][j] += __shfl_xor_sync(kFull, l[nt][j], o2);
+  }
+};
+
+// One 16-key tile held in shared memory at kbase (K) / vbase (V), 128-byte
+// swizzled boxes of 16 rows x 64 d: S^T = K Q^T, masking, online softmax and
+// o^T += V^T P^T.  valid0 / valid1: whether key rows lane/4 and lane/4 + 8 of
+// the tile belong to the range (at least one row of a tile always does).
+template <int D, int NT>
+__device__ __forceinline__ void tc_tile(WarpAcc<D, NT>& acc, const uint32_t (&qf)[NT][D / 16][2],
+                                        uint32_t kbase, uint32_t vbase, bool valid0, bool valid1,
+                                        float scale_log2, int lane) {
+  constexpr int STEPS = D / 16;
+  // ---- S^T = K Q^T (16 keys x 8 heads per n-tile)
+  float sacc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+  {
+    const int r = lane & 15;  // key row of this lane's ldmatrix address
+#pragma unroll
+    for (int ks = 0; ks < STEPS; ++ks) {
+      const int half = ks >> 2;
+      const int chunk = ((ks & 3) << 1) + (lane >> 4);  // 16-byte chunk within the half
+      uint32_t af[4];
+      ldsm_x4(kbase + half * kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), af);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
+    }
+  }
+
+  // ---- mask, online softmax (base 2)
+  float p[NT][4];
+  bool rescale = false;
+  float alpha[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float s0 = valid0 ? sacc[nt][0] * scale_log2 : -INFINITY;
+    const float s1 = valid0 ? sacc[nt][1] * scale_log2 : -INFINITY;
+    const float s2 = valid1 ? sacc[nt][2] * scale_log2 : -INFINITY;
+    const float s3 = valid1 ? sacc[nt][3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+    }
+    // every tile holds at least one valid key, so the new maxima are finite
+    const float mn0 = fmaxf(acc.m[nt][0], mx0), mn1 = fmaxf(acc.m[nt][1], mx1);
+    alpha[nt][0] = exp2f(acc.m[nt][0] - mn0);
+    alpha[nt][1] = exp2f(acc.m[nt][1] - mn1);
+    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    acc.m[nt][0] = mn0;
+    acc.m[nt][1] = mn1;
+    p[nt][0] = exp2f(s0 - mn0);
+    p[nt][1] = exp2f(s1 - mn1);
+    p[nt][2] = exp2f(s2 - mn0);
+    p[nt][3] = exp2f(s3 - mn1);
+    acc.l[nt][0] = fmaf(acc.l[nt][0], alpha[nt][0], p[nt][0] + p[nt][2]);
+    acc.l[nt][1] = fmaf(acc.l[nt][1], alpha[nt][1], p[nt][1] + p[nt][3]);
+  }
+  if (__any_sync(kFull, rescale)) {
+#pragma unroll
+    for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        acc.o[dt][nt][0] *= alpha[nt][0];
+        acc.o[dt][nt][1] *= alpha[nt][1];
+        acc.o[dt][nt][2] *= alpha[nt][0];
+        acc.o[dt][nt][3] *= alpha[nt][1];
+      }
+  }
+
+  // ---- o^T += V^T P^T.  P enters the bf16 product as hi + lo, two bf16
+  // parts whose sum carries ~16 significant bits, so a split of a few keys
+  // with large, opposite V rows keeps fp32-level accuracy.
+  uint32_t pb[NT][2][2];  // [n-tile][hi, lo][keys 0-7, keys 8-15]
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const uint32_t h01 = pack_bf16x2(p[nt][0], p[nt][1]);
+    const uint32_t h23 = pack_bf16x2(p[nt][2], p[nt][3]);
+    const uint32_t l01 = pack_bf16x2(p[nt][0] - bf16lo_to_f32(h01), p[nt][1] - bf16hi_to_f32(h01));
+    const uint32_t l23 = pack_bf16x2(p[nt][2] - bf16lo_to_f32(h23), p[nt][3] - bf16hi_to_f32(h23));
+    pb[nt][0][0] = movmatrix_trans(h01);  // keys 0-7  -> B rows k 0-7
+    pb[nt][0][1] = movmatrix_trans(h23);  // keys 8-15 -> B rows k 8-15
+    pb[nt][1][0] = movmatrix_trans(l01);
+    pb[nt][1][1] = movmatrix_trans(l23);
+  }
+  {
+    const int key = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+    for (int dt = 0; dt < STEPS; ++dt) {
+      const int chunk = dt * 2 + ((lane >> 3) & 1);  // 16-byte chunk along d
+      const int half = chunk >> 3, cc = chunk & 7;
+      uint32_t af[4];
+      ldsm_x4_trans(vbase + half * kBoxBytes + key * 128 + ((cc ^ (key & 7)) << 4), af);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16_16816(acc.o[dt][nt], af, pb[nt][0][0], pb[nt][0][1]);
+        mma_bf16_16816(acc.o[dt][nt], af, pb[nt][1][0], pb[nt][1][1]);
+      }
+    }
+  }
+}
+
+// Issues the TMA loads of one stage: both d halves of K then of V for the
+// 16 rows starting at packed row `row` of kv head g.
+template <int D>
+__device__ __forceinline__ void tc_issue_stage(uint32_t dst, uint32_t bar, const CUtensorMap* kmap,
+                                               const CUtensorMap* vmap, int g, int row,
+                                               uint64_t policy) {
+  constexpr int HALVES = TcShape<D>::kHalves;
+  mbar_arrive_expect_tx(bar, TcShape<D>::kStageBytes);
+#pragma unroll
+  for (int h = 0; h < HALVES; ++h) tma_load_3d(dst + h * kBoxBytes, kmap, h * 64, g, row, bar, policy);
+#pragma unroll
+  for (int h = 0; h < HALVES; ++h)
+    tma_load_3d(dst + (HALVES + h) * kBoxBytes, vmap, h * 64, g, row, bar, policy);
+}
+
+// 1024-byte-aligned start of the dynamic shared memory (128-byte swizzle
+// atoms repeat every 1024 bytes).
+__device__ __forceinline__ uint8_t* aligned_dyn_smem(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                    ~static_cast<uintptr_t>(1023));
+}
+
+// Per-split partial kernel: one CTA per (split, kv head g, head block, b)
+// writes that split's triplet (gqa_decode_partial).
+template <int D, int NT, int NW, int NS>
 __global__ void __launch_bounds__(NW * 32)
     decode_tc_bf16(const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
@@ -62,18 +243,15 @@ __global__ void __launch_bounds__(NW * 32)
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[NW * NS];
   __shared__ float sm_m[NW * HB], sm_l[NW * HB];
-  __shared__ int sm_flag;
 
-  uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~static_cast<uintptr_t>(1023));
-
+  uint8_t* stages = aligned_dyn_smem(dyn_smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = blockIdx.x, b = blockIdx.z;
   const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
   const Split sp = locate_split(a, b, slot, lane,
                                 warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
   if (slot >= sp.n_active) {
-    if (MODE == kPartial) emit_empty_triplet<HB, D>(a, b, g, hb, slot);
+    emit_empty_triplet<HB, D>(a, b, g, hb, slot);
     return;
   }
 
@@ -85,24 +263,6 @@ __global__ void __launch_bounds__(NW * 32)
     fence_barrier_init();
   }
   __syncthreads();
-
-  // Q^T as the B operand of S^T = K Q^T: thread holds head (lane / 4) and
-  // d = 16 * ks + 2 * (lane % 4) + {0, 1} (b0) and + {8, 9} (b1).
-  uint32_t qf[NT][STEPS][2];
-  {
-    const uint32_t* qw = static_cast<const uint32_t*>(a.q);  // bf16 pairs
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int gi = hb * HB + nt * 8 + (lane >> 2);
-      const bool ok = gi < a.G;
-      const size_t base = (query_row(a, b, g, ok ? gi : 0) * D) / 2 + (lane & 3);
-#pragma unroll
-      for (int ks = 0; ks < STEPS; ++ks) {
-        qf[nt][ks][0] = ok ? __ldg(qw + base + ks * 8) : 0u;
-        qf[nt][ks][1] = ok ? __ldg(qw + base + ks * 8 + 4) : 0u;
-      }
-    }
-  }
 
   const int len = sp.hi - sp.lo;
   const int ntiles = (len + KT - 1) / KT;
@@ -116,15 +276,8 @@ __global__ void __launch_bounds__(NW * 32)
     return (ts + KT <= sp.hi) ? ts : sp.hi - KT;
   };
   auto issue = [&](int t, int s) {
-    const uint32_t bar = bar0 + s * 8;
-    const uint32_t dst = stage0 + s * STAGE;
-    const int row = static_cast<int>(sp.off + tile_row0(t));
-    mbar_arrive_expect_tx(bar, STAGE);
-#pragma unroll
-    for (int h = 0; h < HALVES; ++h) tma_load_3d(dst + h * kBoxBytes, &kmap, h * 64, g, row, bar, policy);
-#pragma unroll
-    for (int h = 0; h < HALVES; ++h)
-      tma_load_3d(dst + (HALVES + h) * kBoxBytes, &vmap, h * 64, g, row, bar, policy);
+    tc_issue_stage<D>(stage0 + s * STAGE, bar0 + s * 8, &kmap, &vmap, g,
+                      static_cast<int>(sp.off + tile_row0(t)), policy);
   };
 
   if (lane == 0) {
@@ -136,17 +289,10 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncwarp();
 
-  float m_run[NT][2], l_run[NT][2];
-  float oacc[STEPS][NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-    for (int dt = 0; dt < STEPS; ++dt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) oacc[dt][nt][e] = 0.f;
-  }
+  uint32_t qf[NT][STEPS][2];
+  load_q_frags<D, NT>(qf, a, b, g, hb, lane);
+  WarpAcc<D, NT> acc;
+  acc.reset();
 
   int it = 0;
   bool failed = false;
@@ -159,104 +305,12 @@ __global__ void __launch_bounds__(NW * 32)
       break;
     }
     const uint32_t kbase = stage0 + s * STAGE;
-    const uint32_t vbase = kbase + HALVES * kBoxBytes;
-
-    // ---- S^T = K Q^T (16 keys x 8 heads per n-tile)
-    float sacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-    {
-      const int r = lane & 15;  // key row of this lane's ldmatrix address
-#pragma unroll
-      for (int ks = 0; ks < STEPS; ++ks) {
-        const int half = ks >> 2;
-        const int chunk = ((ks & 3) << 1) + (lane >> 4);  // 16-byte chunk within the half
-        uint32_t af[4];
-        ldsm_x4(kbase + half * kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), af);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], af, qf[nt][ks][0], qf[nt][ks][1]);
-      }
-    }
-
-    // ---- mask, online softmax (base 2)
     const int ts = sp.lo + t * KT;
     const int row0 = tile_row0(t);
-    const bool valid0 = row0 + (lane >> 2) >= ts;      // key row lane/4
-    const bool valid1 = row0 + (lane >> 2) + 8 >= ts;  // key row lane/4 + 8
-    float p[NT][4];
-    bool rescale = false;
-    float alpha[NT][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const float s0 = valid0 ? sacc[nt][0] * a.scale_log2 : -INFINITY;
-      const float s1 = valid0 ? sacc[nt][1] * a.scale_log2 : -INFINITY;
-      const float s2 = valid1 ? sacc[nt][2] * a.scale_log2 : -INFINITY;
-      const float s3 = valid1 ? sacc[nt][3] * a.scale_log2 : -INFINITY;
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
-      }
-      // every tile holds at least one valid key, so the new maxima are finite
-      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-      alpha[nt][0] = exp2f(m_run[nt][0] - mn0);
-      alpha[nt][1] = exp2f(m_run[nt][1] - mn1);
-      rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-      m_run[nt][0] = mn0;
-      m_run[nt][1] = mn1;
-      p[nt][0] = exp2f(s0 - mn0);
-      p[nt][1] = exp2f(s1 - mn1);
-      p[nt][2] = exp2f(s2 - mn0);
-      p[nt][3] = exp2f(s3 - mn1);
-      l_run[nt][0] = fmaf(l_run[nt][0], alpha[nt][0], p[nt][0] + p[nt][2]);
-      l_run[nt][1] = fmaf(l_run[nt][1], alpha[nt][1], p[nt][1] + p[nt][3]);
-    }
-    if (__any_sync(kFull, rescale)) {
-#pragma unroll
-      for (int dt = 0; dt < STEPS; ++dt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          oacc[dt][nt][0] *= alpha[nt][0];
-          oacc[dt][nt][1] *= alpha[nt][1];
-          oacc[dt][nt][2] *= alpha[nt][0];
-          oacc[dt][nt][3] *= alpha[nt][1];
-        }
-    }
-
-    // ---- o^T += V^T P^T.  P enters the bf16 product as hi + lo, two bf16
-    // parts whose sum carries ~16 significant bits, so a split of a few keys
-    // with large, opposite V rows keeps fp32-level accuracy.
-    uint32_t pb[NT][2][2];  // [n-tile][hi, lo][keys 0-7, keys 8-15]
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t h01 = pack_bf16x2(p[nt][0], p[nt][1]);
-      const uint32_t h23 = pack_bf16x2(p[nt][2], p[nt][3]);
-      const uint32_t l01 = pack_bf16x2(p[nt][0] - bf16lo_to_f32(h01), p[nt][1] - bf16hi_to_f32(h01));
-      const uint32_t l23 = pack_bf16x2(p[nt][2] - bf16lo_to_f32(h23), p[nt][3] - bf16hi_to_f32(h23));
-      pb[nt][0][0] = movmatrix_trans(h01);  // keys 0-7  -> B rows k 0-7
-      pb[nt][0][1] = movmatrix_trans(h23);  // keys 8-15 -> B rows k 8-15
-      pb[nt][1][0] = movmatrix_trans(l01);
-      pb[nt][1][1] = movmatrix_trans(l23);
-    }
-    {
-      const int key = (lane & 7) + ((lane >> 4) << 3);
-#pragma unroll
-      for (int dt = 0; dt < STEPS; ++dt) {
-        const int chunk = dt * 2 + ((lane >> 3) & 1);  // 16-byte chunk along d
-        const int half = chunk >> 3, cc = chunk & 7;
-        uint32_t af[4];
-        ldsm_x4_trans(vbase + half * kBoxBytes + key * 128 + ((cc ^ (key & 7)) << 4), af);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_bf16_16816(oacc[dt][nt], af, pb[nt][0][0], pb[nt][0][1]);
-          mma_bf16_16816(oacc[dt][nt], af, pb[nt][1][0], pb[nt][1][1]);
-        }
-      }
-    }
+    tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
+                   row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
     __syncwarp();
-
-    // ---- refill this stage with the warp's tile NS steps ahead
+    // refill this stage with the warp's tile NS steps ahead
     const int tn = t + NS * NW;
     if (lane == 0 && tn < ntiles) {
       fence_proxy_async_smem();
@@ -271,24 +325,9 @@ __global__ void __launch_bounds__(NW * 32)
     const int my_tiles = (ntiles > warp) ? (ntiles - warp + NW - 1) / NW : 0;
     const int last = min(it + NS, my_tiles);
     for (int i = it; i < last; ++i) mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      m_run[nt][0] = m_run[nt][1] = -INFINITY;
-      l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-      for (int dt = 0; dt < STEPS; ++dt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[dt][nt][e] = 0.f;
-    }
+    acc.reset();
   }
-
-  // denominators: sum over the 8 lanes that share a head column
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) l_run[nt][j] += __shfl_xor_sync(kFull, l_run[nt][j], o);
+  acc.reduce_l();
 
   __syncthreads();  // every warp is done with its stages: reuse them for o
   float* sm_o = reinterpret_cast<float*>(stages);
@@ -297,8 +336,8 @@ __global__ void __launch_bounds__(NW * 32)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        sm_m[warp * HB + nt * 8 + 2 * lane + j] = m_run[nt][j];
-        sm_l[warp * HB + nt * 8 + 2 * lane + j] = l_run[nt][j];
+        sm_m[warp * HB + nt * 8 + 2 * lane + j] = acc.m[nt][j];
+        sm_l[warp * HB + nt * 8 + 2 * lane + j] = acc.l[nt][j];
       }
   }
 #pragma unroll
@@ -309,11 +348,10 @@ __global__ void __launch_bounds__(NW * 32)
       for (int e = 0; e < 4; ++e) {
         const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
         const int head = nt * 8 + 2 * (lane & 3) + (e & 1);
-        sm_o[(warp * HB + head) * D + d] = oacc[dt][nt][e];
+        sm_o[(warp * HB + head) * D + d] = acc.o[dt][nt][e];
       }
   __syncthreads();
   emit_split_triplet<NW, HB, D>(sm_m, sm_l, sm_o, a, b, g, hb, slot);
-  if (MODE == kFused) fused_finish<NW, HB, D>(a, b, g, hb, sp.n_active, &sm_flag);
 }
 
 }  // namespace gqa

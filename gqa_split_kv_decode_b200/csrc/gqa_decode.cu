@@ -15,6 +15,7 @@
 
 #include "gqa_decode.h"
 #include "decode_simt.cuh"
+#include "decode_streamk.cuh"
 #include "decode_tc.cuh"
 #include "split_merge.cuh"
 
@@ -116,17 +117,60 @@ int after_launch() {
 constexpr int kTcWarps = GQA_TC_WARPS;
 constexpr int kTcStages = GQA_TC_STAGES;
 
-template <int D, int NT, int MODE>
-int launch_tc(const DecodeArgs& a, const void* k, const void* v, dim3 grid, cudaStream_t st) {
+// Per-split kernel (gqa_decode_partial).
+template <int D, int NT>
+int launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   constexpr int NW = kTcWarps, NS = kTcStages;
   constexpr int smem = tc_dynamic_smem<D, NW, NS>();
   static std::atomic<uint64_t> attr_done{0};
-  auto kern = decode_tc_bf16<D, NT, NW, NS, MODE>;
+  auto kern = decode_tc_bf16<D, NT, NW, NS>;
   if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
   CUtensorMap kmap, vmap;
-  if (!encode_cache_map(&kmap, k, a.h_kv, D) || !encode_cache_map(&vmap, v, a.h_kv, D))
+  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
   kern<<<grid, NW * 32, smem, st>>>(kmap, vmap, a);
+  return after_launch();
+}
+
+// Persistent fused kernel: as many CTAs as fit on the GPU at once (at most
+// kMaxStreamWarps warps in all, which bounds the piece storage).
+constexpr int kMaxStreamWarps = 2048;
+
+int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return -1;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+template <int D, int NT>
+int launch_tc_streamk(const DecodeArgs& a, const PieceStore& ps, cudaStream_t st) {
+  constexpr int NW = kTcWarps, NS = kTcStages;
+  constexpr int smem = tc_dynamic_smem<D, NW, NS>();
+  static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<int> per_sm[kMaxDevices];
+  auto kern = decode_tc_bf16_streamk<D, NT, NW, NS>;
+  if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
+  const int dev = current_device();
+  const int sms = sm_count();
+  if (dev < 0 || sms <= 0) return GQA_ERR_CUDA;
+  int occ = per_sm[dev].load(std::memory_order_relaxed);
+  if (occ <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NW * 32, smem) != cudaSuccess ||
+        occ <= 0)
+      return GQA_ERR_CUDA;
+    per_sm[dev].store(occ, std::memory_order_relaxed);
+  }
+  int ctas = sms * occ;
+  if (ctas * NW > kMaxStreamWarps) ctas = kMaxStreamWarps / NW;
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
+    return GQA_ERR_CUDA;
+  kern<<<ctas, NW * 32, smem, st>>>(kmap, vmap, a, ps);
   return after_launch();
 }
 
@@ -148,21 +192,29 @@ int launch_simt_hb(const DecodeArgs& a, int hb, dim3 grid, cudaStream_t st) {
   }
 }
 
+// bf16 partials or any fp32 work: one CTA per (split, kv head, head block, b).
 template <int MODE>
-int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
+int launch_per_split(DecodeArgs a, int dtype, int D, cudaStream_t st) {
   const int hb = heads_per_cta(dtype, a.G);
   a.n_hb = (a.G + hb - 1) / hb;
   const dim3 grid(a.n_slots, a.h_kv * a.n_hb, a.B);
   if (dtype == GQA_BF16) {
     const bool wide = hb == 16;
-    if (D == 128)
-      return wide ? launch_tc<128, 2, MODE>(a, a.k, a.v, grid, st)
-                  : launch_tc<128, 1, MODE>(a, a.k, a.v, grid, st);
-    return wide ? launch_tc<64, 2, MODE>(a, a.k, a.v, grid, st)
-                : launch_tc<64, 1, MODE>(a, a.k, a.v, grid, st);
+    if (D == 128) return wide ? launch_tc<128, 2>(a, grid, st) : launch_tc<128, 1>(a, grid, st);
+    return wide ? launch_tc<64, 2>(a, grid, st) : launch_tc<64, 1>(a, grid, st);
   }
   if (D == 128) return launch_simt_hb<128, MODE>(a, hb, grid, st);
   return launch_simt_hb<64, MODE>(a, hb, grid, st);
+}
+
+// Fused bf16: the persistent even-split kernel.
+int launch_fused_bf16(DecodeArgs a, const PieceStore& ps, int D, cudaStream_t st) {
+  const int hb = tc_heads_per_cta(a.G);
+  a.n_hb = (a.G + hb - 1) / hb;
+  const bool wide = hb == 16;
+  if (D == 128)
+    return wide ? launch_tc_streamk<128, 2>(a, ps, st) : launch_tc_streamk<128, 1>(a, ps, st);
+  return wide ? launch_tc_streamk<64, 2>(a, ps, st) : launch_tc_streamk<64, 1>(a, ps, st);
 }
 
 // ------------------------------------------------------------ validation
@@ -248,7 +300,8 @@ size_t n_tickets(const Shape& s) {
   return (size_t)s.B * s.h_kv * (G <= 16 ? 1 : (G + 15) / 16);
 }
 
-WsLayout ws_layout(const Shape& s) {
+// fp32 fused path: one triplet per (b, h, split).
+WsLayout ws_layout_triplets(const Shape& s) {
   const size_t rows = (size_t)s.B * s.h_q;
   WsLayout w;
   w.tickets = 0;
@@ -257,6 +310,45 @@ WsLayout ws_layout(const Shape& s) {
   w.o = w.l + round_up(rows * s.n_slots * sizeof(float), 256);
   w.total = w.o + round_up(rows * s.n_slots * s.D * sizeof(float), 256);
   return w;
+}
+
+// bf16 fused path: pieces, one per (unit, warp) pair that meet; at most
+// (non-empty units) + (warps) of them, each holding min(16, G) heads.
+int piece_heads(const Shape& s) {
+  const int G = s.h_q / s.h_kv;
+  const int hb = tc_heads_per_cta(G);
+  return G < hb ? G : hb;
+}
+
+size_t piece_slots(const Shape& s) {
+  const int G = s.h_q / s.h_kv;
+  const int hb = tc_heads_per_cta(G);
+  const size_t units = (size_t)s.B * s.h_kv * ((G + hb - 1) / hb) * s.n_slots;
+  return units + kMaxStreamWarps;
+}
+
+WsLayout ws_layout_pieces(const Shape& s) {
+  const size_t cells = piece_slots(s) * piece_heads(s);
+  WsLayout w;
+  w.tickets = 0;
+  w.m = kTicketBytes;
+  w.l = w.m + round_up(cells * sizeof(float), 256);
+  w.o = w.l + round_up(cells * sizeof(float), 256);
+  w.total = w.o + round_up(cells * s.D * sizeof(float), 256);
+  return w;
+}
+
+WsLayout ws_layout(const Shape& s) {
+  return s.dtype == GQA_BF16 ? ws_layout_pieces(s) : ws_layout_triplets(s);
+}
+
+// Bytes that serve either dtype (the size queries take no dtype).
+size_t ws_bytes_any_dtype(Shape s) {
+  s.dtype = GQA_BF16;
+  const size_t a = ws_layout(s).total;
+  s.dtype = GQA_F32;
+  const size_t b = ws_layout(s).total;
+  return a > b ? a : b;
 }
 
 struct LibWorkspace {
@@ -309,11 +401,19 @@ int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, f
   DecodeArgs a = make_args(q, k, v, seqlens, s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   a.tickets = reinterpret_cast<int*>(base + w.tickets);
+  a.out = out;
+  if (s.dtype == GQA_BF16) {
+    PieceStore ps;
+    ps.m = reinterpret_cast<float*>(base + w.m);
+    ps.l = reinterpret_cast<float*>(base + w.l);
+    ps.o = reinterpret_cast<float*>(base + w.o);
+    ps.HBs = piece_heads(s);
+    return launch_fused_bf16(a, ps, s.D, as_stream(stream));
+  }
   a.m = reinterpret_cast<float*>(base + w.m);
   a.l = reinterpret_cast<float*>(base + w.l);
   a.o = reinterpret_cast<float*>(base + w.o);
-  a.out = out;
-  return launch_decode<kFused>(a, s.dtype, s.D, as_stream(stream));
+  return launch_per_split<kFused>(a, s.dtype, s.D, as_stream(stream));
 }
 
 int partial(const void* q, const void* k, const void* v, const int32_t* seqlens, float* m,
@@ -326,7 +426,7 @@ int partial(const void* q, const void* k, const void* v, const int32_t* seqlens,
   a.m = m;
   a.l = l;
   a.o = o;
-  return launch_decode<kPartial>(a, s.dtype, s.D, as_stream(stream));
+  return launch_per_split<kPartial>(a, s.dtype, s.D, as_stream(stream));
 }
 
 __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
@@ -365,14 +465,14 @@ const char* gqa_decode_error_string(int status) {
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits) {
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, 1.f, GQA_BF16);
   if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
-  return ws_layout(s).total;
+  return ws_bytes_any_dtype(s);
 }
 
 size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head, int chunk_len,
                                          int max_seqlen) {
   const Shape s = chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, 1.f, GQA_BF16);
   if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
-  return ws_layout(s).total;
+  return ws_bytes_any_dtype(s);
 }
 
 int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,

@@ -104,16 +104,25 @@ def test_partial_and_merge_argument_checks(lib):
 
 
 def test_workspace_size_arithmetic(lib):
-    # fixed 256 KiB ticket area + m + l (B*h_q*n fp32 each) + o (B*h_q*n*d fp32), 256-byte rounded
-    B, hq, hkv, d, n = 8, 64, 8, 128, 8
+    """Fixed 256 KiB ticket area, then the larger of the two fused layouts:
+    fp32 triplets (m, l, o for every (b, h, split)) or bf16 pieces (one per
+    (unit, warp) pair that meet: at most units + 2048, min(16, G) heads each)."""
     r = lambda x: (x + 255) // 256 * 256
     T = 256 * 1024
-    expect = T + 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
-    assert lib.gqa_decode_workspace_size(B, hq, hkv, d, n) == expect
-    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == T + 2 * r(32 * 2 * 4) + r(32 * 2 * 128 * 4)
-    assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == \
-        T + 2 * r(64 * 32 * 32 * 4) + r(64 * 32 * 32 * 128 * 4)
-    # more than 65536 tickets (B * h_kv * head blocks) is refused
-    assert lib.gqa_decode_workspace_size(65535, 8, 2, 128, 1) == 0
+
+    def expect(B, hq, hkv, d, n):
+        G = hq // hkv
+        trip = 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
+        blocks = 1 if G <= 16 else -(-G // 16)
+        cells = (B * hkv * blocks * n + 2048) * min(G, 8 if G <= 8 else 16)
+        pieces = 2 * r(cells * 4) + r(cells * d * 4)
+        return T + max(trip, pieces)
+
+    assert lib.gqa_decode_workspace_size(8, 64, 8, 128, 8) == expect(8, 64, 8, 128, 8)
+    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == expect(1, 32, 1, 128, 2)
+    assert lib.gqa_decode_workspace_size(64, 32, 8, 128, 3) == expect(64, 32, 8, 128, 3)
+    assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == expect(64, 32, 8, 128, 32)
     assert lib.gqa_decode_workspace_size(1, 6, 4, 128, 4) == 0
     assert lib.gqa_decode_workspace_size(1, 8, 2, 96, 4) == 0
+    # more than 65536 tickets (B * h_kv * head blocks) is refused
+    assert lib.gqa_decode_workspace_size(65535, 8, 2, 128, 1) == 0

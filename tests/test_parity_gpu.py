@@ -235,14 +235,21 @@ def test_dominant_logit_and_large_values(gk):
 
 # ------------------------------------------------------- exactness properties
 
-def test_fused_equals_partial_then_merge_bitwise(gk):
-    w = workloads.generate(scaled("llama70b", B=2, S=3000))
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fused_matches_partial_then_merge(gk, dtype):
+    """The fused call and partial + mlo_merge are two groupings of the same
+    exact merge: they agree to fp32 rounding (bitwise on the fp32 path,
+    which shares the per-split kernel)."""
+    w = random_case(3, 64, 8, 128, [3000, 17, 900], dtype=dtype, seed=40)
     c = w.cfg
     q, k, v, sl = dev(w)
     fused = gk.gqa_decode_attn(q, k, v, sl, 8, c.scale)
     m, l, o = gk.gqa_decode_partial(q, k, v, sl, 8, c.scale)
     merged = gk.mlo_merge(m, l, o)
-    assert torch.equal(fused, merged)
+    if dtype == "f32":
+        assert torch.equal(fused, merged)
+    else:
+        assert torch.allclose(fused, merged, atol=1e-5, rtol=1e-4)
 
 
 def test_deterministic_and_workspace_reuse(gk):
