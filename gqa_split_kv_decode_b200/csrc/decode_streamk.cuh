@@ -1,22 +1,27 @@
 // Fused bf16 decode attention with an even, persistent split of the work.
 //
-// The work is the sequence of 16-key tiles of every unit u = (b, kv head /
-// head block gy, split slot), in that order (T tiles in all).  The grid holds
-// exactly the CTAs that fit on the GPU at once; its Wv = min(warps, T) warps
-// each take one contiguous run of tiles [w*T/Wv, (w+1)*T/Wv), so every warp
-// streams the same number of bytes and no second wave starts cold.  A warp
-// keeps its TMA ring running across unit boundaries and emits one partial
-// triplet (a "piece", kernbench "_attention_mesh_mlo.py": "One-shot local
-// partial attention" over the keys it saw) for each unit it touches; a piece
-// never spans two splits, so the user's split structure is preserved.  The
-// pieces of a group (b, gy) are merged with the page's log-sum-exp rule by
-// the warp that completes the group's last tile (a per-group counter of
-// finished tiles, incremented once per piece; nothing waits on another
-// warp), which also normalises and writes out.
+// Every kv head (head block) gy sees the same sequence of 16-key tiles: the
+// tiles of every unit (b, split), in that order, T1 tiles in all.  The grid
+// holds exactly the CTAs that fit on the GPU at once.  Its warps are laid out
+// head-minor: warp w serves head gy = w % H and takes run k = w / H of that
+// head's tiles, [k*T1/Wk, (k+1)*T1/Wk), so every warp streams the same number
+// of bytes, no second wave starts cold, and the warps that share k (the four
+// warps of a CTA, and their neighbours) read the same cache rows of
+// different kv heads together -- a cache row holds every kv head's keys side
+// by side, so that keeps DRAM pages open.  A warp keeps its TMA ring running
+// across unit boundaries and emits one partial triplet (a "piece",
+// kernbench "_attention_mesh_mlo.py": "One-shot local partial attention" over
+// the keys it saw) for each unit it touches; a piece never spans two splits,
+// so the user's split structure is preserved.  The pieces of a group (b, gy)
+// are merged with the page's log-sum-exp rule by the warp that completes the
+// group's last tile (a per-group counter of finished tiles, incremented once
+// per piece; nothing waits on another warp), which also normalises and
+// writes out.
 //
-// Piece storage: piece (u, w) exists iff warp w's run meets unit u; ordered
-// by tile position each next piece increments u, w or both, so u + w is a
-// unique slot in [0, U + Wv) (U = number of non-empty units).
+// Piece storage: within head gy, piece (u, k) exists iff run k meets unit u;
+// ordered by tile position each next piece increments u, k or both, so
+// u + k is unique in [0, U1 + Wk) (U1 = non-empty units per head) and piece
+// (gy, u, k) lives at slot gy * (U1 + Wk) + u + k.
 #pragma once
 
 #include "decode_tc.cuh"
@@ -59,12 +64,12 @@ __device__ __forceinline__ int tiles_in(const SeqGeom& q, int slot) {
   return slot == q.n_act - 1 ? q.tlast : q.tps;
 }
 
-// Position of a warp in the tile sequence (identical in every lane).
+// Position of a warp in its head's tile sequence (identical in every lane).
 struct Cursor {
-  int b, gy, slot, tile;
+  int b, slot, tile;
   long long off;  // packed row of sequence b's first key
-  long long F;    // tile index of (b, gy 0, split 0, tile 0)
-  long long U;    // unit index of (b, gy 0, split 0)
+  long long F;    // per-head tile index of (b, split 0, tile 0)
+  long long U;    // per-head unit index of (b, split 0)
   SeqGeom q;
 };
 
@@ -77,14 +82,14 @@ __device__ __forceinline__ long long scan_incl(long long v, int lane) {
   return v;
 }
 
-// Cursor at tile t0 (0 <= t0 < T).  Whole warp.
-__device__ Cursor locate_tile(const DecodeArgs& a, int H, long long t0, int lane) {
+// Cursor at per-head tile t0 (0 <= t0 < T1).  Whole warp.
+__device__ Cursor locate_tile(const DecodeArgs& a, long long t0, int lane) {
   long long F = 0, U = 0, off = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
     const int S = b < a.B ? __ldg(a.seqlens + b) : 0;
     const SeqGeom q = seq_geom(a, S);
-    const long long tiles = (long long)H * q.Tg, units = (long long)H * q.n_act, rows = q.S;
+    const long long tiles = q.Tg, units = q.n_act, rows = q.S;
     const long long ti = scan_incl(tiles, lane), ui = scan_incl(units, lane), ri = scan_incl(rows, lane);
     const unsigned hit = __ballot_sync(kFull, F + ti > t0);
     if (hit) {
@@ -95,9 +100,7 @@ __device__ Cursor locate_tile(const DecodeArgs& a, int H, long long t0, int lane
       c.U = U + __shfl_sync(kFull, ui - units, j);
       c.off = off + __shfl_sync(kFull, ri - rows, j);
       c.q = seq_geom(a, __shfl_sync(kFull, S, j));
-      const long long local = t0 - c.F;
-      c.gy = (int)(local / c.q.Tg);
-      const int r = (int)(local - (long long)c.gy * c.q.Tg);
+      const int r = (int)(t0 - c.F);
       int slot = r / c.q.tps;
       if (slot > c.q.n_act - 1) slot = c.q.n_act - 1;
       c.slot = slot;
@@ -108,20 +111,18 @@ __device__ Cursor locate_tile(const DecodeArgs& a, int H, long long t0, int lane
     U += __shfl_sync(kFull, ui, 31);
     off += __shfl_sync(kFull, ri, 31);
   }
-  Cursor none{};  // not reached for t0 < T
+  Cursor none{};  // not reached for t0 < T1
   return none;
 }
 
 // Moves the cursor to the next tile; the caller guarantees one exists.
-__device__ __forceinline__ void advance(Cursor& c, const DecodeArgs& a, int H) {
+__device__ __forceinline__ void advance(Cursor& c, const DecodeArgs& a) {
   if (++c.tile < tiles_in(c.q, c.slot)) return;
   c.tile = 0;
   if (++c.slot < c.q.n_act) return;
   c.slot = 0;
-  if (++c.gy < H) return;
-  c.gy = 0;
-  c.F += (long long)H * c.q.Tg;
-  c.U += (long long)H * c.q.n_act;
+  c.F += c.q.Tg;
+  c.U += c.q.n_act;
   c.off += c.q.S;
   for (;;) {  // skip empty sequences (they add no rows, tiles or units)
     ++c.b;
@@ -154,17 +155,18 @@ struct PieceStore {
   int HBs;    // heads stored per piece = min(HB, G)
 };
 
-// Merges every piece of group (b, gy) in split and warp order, normalises,
+// Merges every piece of group (b, gy) in split and run order, normalises,
 // and writes the group's rows of out.  Whole warp.
 template <int D, int NT>
 __device__ __noinline__ void merge_group(const DecodeArgs& a, const PieceStore ps, int b, int gy,
-                                         SeqGeom q, long long Fb, long long Ub, long long T,
-                                         long long Wv, int lane) {
+                                         SeqGeom q, long long Fb, long long Ub, long long T1,
+                                         long long Wk, long long U1, int lane) {
   constexpr int HB = NT * 8;
   constexpr int PER = D / 32;  // contiguous elements of d per lane
   const int g = gy / a.n_hb, hb = gy % a.n_hb;
-  const long long Fg = Fb + (long long)gy * q.Tg;
-  const long long Ug = Ub + (long long)gy * q.n_act;
+  const long long Fg = Fb;
+  const long long Ug = (long long)gy * (U1 + Wk) + Ub;
+  const long long T = T1, Wv = Wk;
   const int HBs = ps.HBs;
 
   float M[HB];
@@ -269,8 +271,9 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncthreads();  // the only CTA-wide barrier: warps run independently from here
 
-  // Total tiles; rows of empty sequences are written (zeros) by warp b % W.
-  long long T = 0;
+  // Per-head tiles T1 and units U1; rows of empty sequences are written
+  // (zeros) by warp b % W.
+  long long T1 = 0, U1 = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
     const int S = b < a.B ? __ldg(a.seqlens + b) : 0;
@@ -279,7 +282,8 @@ __global__ void __launch_bounds__(NW * 32)
     if (wid == 0 && b < a.B && a.chunk_len > 0 &&
         (long long)q.S > (long long)a.n_slots * a.chunk_len)
       raise_status(kStatusSeqlenOverMax);
-    T += __shfl_sync(kFull, scan_incl((long long)H * q.Tg, lane), 31);
+    T1 += __shfl_sync(kFull, scan_incl(q.Tg, lane), 31);
+    U1 += __shfl_sync(kFull, scan_incl(q.n_act, lane), 31);
     unsigned empty = __ballot_sync(kFull, b < a.B && q.S == 0 && (b % W) == wid);
     while (empty) {
       const int j = __ffs(empty) - 1;
@@ -288,116 +292,127 @@ __global__ void __launch_bounds__(NW * 32)
       for (int i = lane; i < a.h_q * D; i += 32) dst[i] = 0.f;
     }
   }
-  if (T == 0) return;
-  const long long Wv = T < W ? T : W;
-  if (wid >= Wv) return;
-  const long long t0 = wid * T / Wv, t1 = (wid + 1) * T / Wv;
+  if (T1 == 0) return;
+  long long Wg = W / H;
+  if (Wg < 1) Wg = 1;
+  const long long Wk = T1 < Wg ? T1 : Wg;  // runs per head
 
   const uint64_t policy = l2_policy_evict_first();
   const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
   const uint32_t bar0 = smem_u32(&full_bar[warp * NS]);
+  uint32_t phase_base = 0;  // uses of this warp's stages so far (for mbarrier parity)
 
-  Cursor cc = locate_tile(a, H, t0, lane);  // tile being computed
-  Cursor ic = cc;                           // next tile to load
-  auto issue = [&](const Cursor& c, int s) {
-    int ts, row0;
-    tile_rows(c, ts, row0);
-    tc_issue_stage<D>(stage0 + s * STAGE, bar0 + s * 8, &kmap, &vmap, c.gy / a.n_hb,
-                      static_cast<int>(c.off + row0), policy);
-  };
-  const long long n_pro = (t1 - t0) < NS ? (t1 - t0) : NS;
-  for (int s = 0; s < n_pro; ++s) {
-    if (lane == 0) issue(ic, s);
-    if (t0 + s + 1 < t1) advance(ic, a, H);
-  }
-  __syncwarp();
+  // Virtual warps vw = wid, wid + W, ... (more than one only when H > W).
+  for (long long vw = wid; vw < Wg * H; vw += W) {
+    const int gy = (int)(vw % H);
+    const long long k = vw / H;
+    if (k >= Wk) continue;
+    const long long t0 = k * T1 / Wk, t1 = (k + 1) * T1 / Wk;
+    const int g = gy / a.n_hb, hb = gy % a.n_hb;
 
-  uint32_t qf[NT][STEPS][2];
-  load_q_frags<D, NT>(qf, a, cc.b, cc.gy / a.n_hb, cc.gy % a.n_hb, lane);
-  WarpAcc<D, NT> acc;
-  acc.reset();
-  int piece_tiles = 0;
-
-  long long it = 0;
-  for (long long t = t0; t < t1; ++t, ++it) {
-    const int s = (int)(it % NS);
-    const uint32_t parity = (uint32_t)((it / NS) & 1);
-    const bool ok = mbar_wait_bounded(bar0 + s * 8, parity, a.timeout_ns);
-    if (!__all_sync(kFull, ok)) {
-      // Record the error, let this warp's issued loads land (bounded), stop.
-      if (lane == 0) raise_status(kStatusTimeout);
-      const long long last = (it + NS < t1 - t0) ? it + NS : t1 - t0;
-      for (long long i = it; i < last; ++i)
-        mbar_wait_bounded(bar0 + (int)(i % NS) * 8, (uint32_t)((i / NS) & 1), a.timeout_ns);
-      return;
+    Cursor cc = locate_tile(a, t0, lane);  // tile being computed
+    Cursor ic = cc;                        // next tile to load
+    auto issue = [&](const Cursor& c, int s) {
+      int ts, row0;
+      tile_rows(c, ts, row0);
+      tc_issue_stage<D>(stage0 + s * STAGE, bar0 + s * 8, &kmap, &vmap, g,
+                        static_cast<int>(c.off + row0), policy);
+    };
+    const long long n_pro = (t1 - t0) < NS ? (t1 - t0) : NS;
+    for (int i = 0; i < n_pro; ++i) {
+      if (lane == 0) issue(ic, (int)((phase_base + i) % NS));
+      if (t0 + i + 1 < t1) advance(ic, a);
     }
-    int ts, row0;
-    tile_rows(cc, ts, row0);
-    const uint32_t kbase = stage0 + s * STAGE;
-    tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
-                   row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
-    ++piece_tiles;
     __syncwarp();
-    // refill this stage with the tile NS ahead
-    if (t + NS < t1) {
-      if (lane == 0) {
-        fence_proxy_async_smem();
-        issue(ic, s);
-      }
-      if (t + NS + 1 < t1) advance(ic, a, H);
-    }
 
-    const bool range_end = (t + 1 == t1);
-    if (range_end || cc.tile + 1 == tiles_in(cc.q, cc.slot)) {
-      // ---- this warp's piece of unit (b, gy, slot) is complete
-      acc.reduce_l();
-      const long long P = cc.U + (long long)cc.gy * cc.q.n_act + cc.slot + wid;
-      const int HBs = ps.HBs;
-      if (lane < 4) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int h = nt * 8 + 2 * lane + j;
-            if (h < HBs) {
-              ps.m[P * HBs + h] = acc.m[nt][j];
-              ps.l[P * HBs + h] = acc.l[nt][j];
-            }
-          }
+    uint32_t qf[NT][STEPS][2];
+    load_q_frags<D, NT>(qf, a, cc.b, g, hb, lane);
+    WarpAcc<D, NT> acc;
+    acc.reset();
+    int piece_tiles = 0;
+
+    for (long long t = t0; t < t1; ++t) {
+      const uint32_t use = phase_base + (uint32_t)(t - t0);
+      const int s = (int)(use % NS);
+      const uint32_t parity = (use / NS) & 1;
+      const bool ok = mbar_wait_bounded(bar0 + s * 8, parity, a.timeout_ns);
+      if (!__all_sync(kFull, ok)) {
+        // Record the error, let this warp's issued loads land (bounded), stop.
+        if (lane == 0) raise_status(kStatusTimeout);
+        const uint32_t end = phase_base + (uint32_t)(t1 - t0);
+        const uint32_t last = (use + NS < end) ? use + NS : end;
+        for (uint32_t i = use; i < last; ++i)
+          mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
+        return;
       }
-#pragma unroll
-      for (int dt = 0; dt < STEPS; ++dt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int h = nt * 8 + 2 * (lane & 3) + (e & 1);
-            const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
-            if (h < HBs) ps.o[(P * HBs + h) * D + d] = acc.o[dt][nt][e];
-          }
-      __threadfence();
+      int ts, row0;
+      tile_rows(cc, ts, row0);
+      const uint32_t kbase = stage0 + s * STAGE;
+      tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
+                     row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
+      ++piece_tiles;
       __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        int* ticket = a.tickets + (size_t)cc.b * H + cc.gy;
-        const int prev = atomicAdd(ticket, piece_tiles);
-        last = (prev + piece_tiles == cc.q.Tg);
-        if (last) atomicExch(ticket, 0);
+      // refill this stage with the tile NS ahead
+      if (t + NS < t1) {
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          issue(ic, s);
+        }
+        if (t + NS + 1 < t1) advance(ic, a);
       }
-      last = __shfl_sync(kFull, last, 0);
-      if (last) {
+
+      const bool range_end = (t + 1 == t1);
+      if (range_end || cc.tile + 1 == tiles_in(cc.q, cc.slot)) {
+        // ---- this warp's piece of unit (b, gy, slot) is complete
+        acc.reduce_l();
+        const long long P = (long long)gy * (U1 + Wk) + cc.U + cc.slot + k;
+        const int HBs = ps.HBs;
+        if (lane < 4) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int h = nt * 8 + 2 * lane + j;
+              if (h < HBs) {
+                ps.m[P * HBs + h] = acc.m[nt][j];
+                ps.l[P * HBs + h] = acc.l[nt][j];
+              }
+            }
+        }
+#pragma unroll
+        for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int h = nt * 8 + 2 * (lane & 3) + (e & 1);
+              const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
+              if (h < HBs) ps.o[(P * HBs + h) * D + d] = acc.o[dt][nt][e];
+            }
         __threadfence();
-        merge_group<D, NT>(a, ps, cc.b, cc.gy, cc.q, cc.F, cc.U, T, Wv, lane);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          int* ticket = a.tickets + (size_t)cc.b * H + gy;
+          const int prev = atomicAdd(ticket, piece_tiles);
+          last = (prev + piece_tiles == cc.q.Tg);
+          if (last) atomicExch(ticket, 0);
+        }
+        last = __shfl_sync(kFull, last, 0);
+        if (last) {
+          __threadfence();
+          merge_group<D, NT>(a, ps, cc.b, gy, cc.q, cc.F, cc.U, T1, Wk, U1, lane);
+        }
+        acc.reset();
+        piece_tiles = 0;
       }
-      acc.reset();
-      piece_tiles = 0;
+      if (!range_end) {
+        const int b_prev = cc.b;
+        advance(cc, a);
+        if (cc.b != b_prev) load_q_frags<D, NT>(qf, a, cc.b, g, hb, lane);
+      }
     }
-    if (!range_end) {
-      const int b_prev = cc.b, gy_prev = cc.gy;
-      advance(cc, a, H);
-      if (cc.b != b_prev || cc.gy != gy_prev)
-        load_q_frags<D, NT>(qf, a, cc.b, cc.gy / a.n_hb, cc.gy % a.n_hb, lane);
-    }
+    phase_base += (uint32_t)(t1 - t0);
   }
 }
 

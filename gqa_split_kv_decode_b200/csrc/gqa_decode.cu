@@ -312,8 +312,9 @@ WsLayout ws_layout_triplets(const Shape& s) {
   return w;
 }
 
-// bf16 fused path: pieces, one per (unit, warp) pair that meet; at most
-// (non-empty units) + (warps) of them, each holding min(16, G) heads.
+// bf16 fused path: pieces, one per (unit, run) pair that meet; at most
+// (non-empty units) + max(warps, kv heads x head blocks) of them, each
+// holding min(16, G) heads.
 int piece_heads(const Shape& s) {
   const int G = s.h_q / s.h_kv;
   const int hb = tc_heads_per_cta(G);
@@ -323,8 +324,9 @@ int piece_heads(const Shape& s) {
 size_t piece_slots(const Shape& s) {
   const int G = s.h_q / s.h_kv;
   const int hb = tc_heads_per_cta(G);
-  const size_t units = (size_t)s.B * s.h_kv * ((G + hb - 1) / hb) * s.n_slots;
-  return units + kMaxStreamWarps;
+  const size_t heads = (size_t)s.h_kv * ((G + hb - 1) / hb);
+  const size_t units = (size_t)s.B * heads * s.n_slots;
+  return units + (heads > (size_t)kMaxStreamWarps ? heads : (size_t)kMaxStreamWarps);
 }
 
 WsLayout ws_layout_pieces(const Shape& s) {
