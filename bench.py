@@ -204,7 +204,7 @@ def run_ours(args, rank, world, local_rank):
     cfg = workloads.CONFIGS[args.config]
     w = workloads.generate(cfg)
     kv_bytes = w.kv_bytes
-    n_copies = max(1, math.ceil(ROTATE_TOTAL / kv_bytes)) if kv_bytes < 2 * L2_BYTES else 1
+    n_copies = max(1, math.ceil(ROTATE_TOTAL / kv_bytes))
     q = w.q.to(device)
     sl = w.seqlens.to(device)
     ks = [w.k.to(device) for _ in range(n_copies)]
@@ -235,31 +235,40 @@ def run_ours(args, rank, world, local_rank):
         time.sleep(0.6)  # let the sampler start before the timed region
 
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize(device)
     sampler.mark_begin()
+    t_start.record(stream)
     for i in range(K):
-        starts[i].record(stream)
         call(i)
-        ends[i].record(stream)
+    t_end.record(stream)
     torch.cuda.synchronize(device)
     sampler.mark_end()
     if world > 1:
         dist.barrier()
-    total_ms = starts[0].elapsed_time(ends[-1])
-    per_launch_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+    total_ms = t_start.elapsed_time(t_end)
     status = gk.get_status(device)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
     sampler.stop()
     clocks = sampler.summary() if rank == 0 else None
 
+    # one launch at a time (events around each call; no overlap between calls)
+    n_iso = min(K, 200)
+    iso_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_iso)]
+    iso_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_iso)]
+    for i in range(n_iso):
+        iso_s[i].record(stream)
+        call(i)
+        iso_e[i].record(stream)
+    torch.cuda.synchronize(device)
+    iso_ms = float(np.median([a.elapsed_time(b) for a, b in zip(iso_s, iso_e)]))
+
     max_total_ms = max_over_ranks(total_ms, world, device)
-    max_launch_ms = max_over_ranks(per_launch_ms, world, device)
+    max_iso_ms = max_over_ranks(iso_ms, world, device)
     all_bytes = sum_over_ranks(float(kv_bytes) * K, world, device)
 
     # ---- end to end through the public API: pinned host inputs in, result out
@@ -304,7 +313,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_src = measured_hbm_peak()
     ms_per_step = max_total_ms / K
     value = all_bytes / (max_total_ms * 1e-3) / 1e9
-    achieved = kv_bytes / (max_launch_ms * 1e-3) / 1e9
+    achieved = kv_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -341,7 +350,9 @@ def run_ours(args, rank, world, local_rank):
             "traffic": profiled_traffic(cfg.name),
             "algorithmic_bytes_per_launch": kv_bytes,
             "kernel": "decode_tc_bf16 (fused, one launch per step)" if cfg.dtype == "bf16" else "decode_simt_f32",
-            "launch_ms": round(max_launch_ms, 6),
+            "timing": "CUDA events around the K back-to-back launches of the timed region",
+            "launch_ms": round(ms_per_step, 6),
+            "isolated_launch_ms": round(max_iso_ms, 6),
         },
         "e2e": {
             "value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 3),

@@ -22,6 +22,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = blockIdx.x, b = blockIdx.z;
   const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
+  grid_dependency_wait();
+  allow_dependent_launch();
   const Split sp = locate_split(a, b, slot, lane,
                                 warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
   if (slot >= sp.n_active) {

@@ -1,10 +1,6 @@
 // bf16 decode attention: TMA-fed K/V tiles, tensor-core logits and PV.
 //
-// This file holds the per-tile math shared by both bf16 kernels and the
-// per-split kernel behind gqa_decode_partial; the fused kernel, which spreads
-// the same tiles evenly over persistent warps, is in decode_streamk.cuh.
-//
-// Per-split kernel: one CTA owns one (split, kv head g, head block, b).  Each of its NW warps
+// One CTA owns one (split, kv head g, head block, b).  Each of its NW warps
 // runs its own NS-stage TMA ring: a stage holds KT = 16 consecutive keys of K
 // and V for kv head g (one 64-element, 128-byte-swizzled box per half of
 // d_head), loaded once from HBM and shared by every query head of the group
@@ -225,9 +221,9 @@ __device__ __forceinline__ uint8_t* aligned_dyn_smem(uint8_t* p) {
                                     ~static_cast<uintptr_t>(1023));
 }
 
-// Per-split partial kernel: one CTA per (split, kv head g, head block, b)
-// writes that split's triplet (gqa_decode_partial).
-template <int D, int NT, int NW, int NS>
+// One CTA per (split, kv head g, head block, b) writes that split's triplet;
+// fused, the CTA that finishes a (b, g, head block) last merges its splits.
+template <int D, int NT, int NW, int NS, int MODE>
 __global__ void __launch_bounds__(NW * 32)
     decode_tc_bf16(const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
@@ -243,17 +239,12 @@ __global__ void __launch_bounds__(NW * 32)
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[NW * NS];
   __shared__ float sm_m[NW * HB], sm_l[NW * HB];
+  __shared__ int sm_flag;
 
   uint8_t* stages = aligned_dyn_smem(dyn_smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = blockIdx.x, b = blockIdx.z;
   const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
-  const Split sp = locate_split(a, b, slot, lane,
-                                warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
-  if (slot >= sp.n_active) {
-    emit_empty_triplet<HB, D>(a, b, g, hb, slot);
-    return;
-  }
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&kmap);
@@ -262,7 +253,16 @@ __global__ void __launch_bounds__(NW * 32)
     for (int i = 0; i < NW * NS; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
     fence_barrier_init();
   }
+  grid_dependency_wait();
+  allow_dependent_launch();
   __syncthreads();
+
+  const Split sp = locate_split(a, b, slot, lane,
+                                warp == 0 && lane == 0 && slot == 0 && blockIdx.y == 0);
+  if (slot >= sp.n_active) {
+    if (MODE == kPartial) emit_empty_triplet<HB, D>(a, b, g, hb, slot);
+    return;
+  }
 
   const int len = sp.hi - sp.lo;
   const int ntiles = (len + KT - 1) / KT;
@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(NW * 32)
       }
   __syncthreads();
   emit_split_triplet<NW, HB, D>(sm_m, sm_l, sm_o, a, b, g, hb, slot);
+  if (MODE == kFused) fused_finish<NW, HB, D>(a, b, g, hb, sp.n_active, &sm_flag);
 }
 
 }  // namespace gqa

@@ -36,6 +36,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ----------------------------------------------- programmatic dependent launch
+
+// Blocks until the grids this launch depends on have completed and their
+// memory is visible (a no-op for an ordinary launch).  Must precede the first
+// read or write of memory another kernel may touch.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next kernel of the stream, if launched with programmatic stream
+// serialization, start its launch now (it still waits for this grid's end
+// before touching memory).
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

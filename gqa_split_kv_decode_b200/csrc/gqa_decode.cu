@@ -12,10 +12,10 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "gqa_decode.h"
 #include "decode_simt.cuh"
-#include "decode_streamk.cuh"
 #include "decode_tc.cuh"
 #include "split_merge.cuh"
 
@@ -104,6 +104,30 @@ int after_launch() {
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// Launches with programmatic stream serialization: the kernel may begin
+// launching while the previous kernel of the stream drains; every kernel
+// here waits for its prerequisites (griddepcontrol.wait) before it touches
+// global memory, so results do not depend on what precedes it.
+template <typename... Params, typename... Args>
+int launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  return after_launch();
+}
+
 // ---------------------------------------------------------- kernel dispatch
 
 // Tensor-core kernel shape: NW warps per CTA, NS stages per warp (build-time
@@ -117,68 +141,23 @@ int after_launch() {
 constexpr int kTcWarps = GQA_TC_WARPS;
 constexpr int kTcStages = GQA_TC_STAGES;
 
-// Per-split kernel (gqa_decode_partial).
-template <int D, int NT>
+template <int D, int NT, int MODE>
 int launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   constexpr int NW = kTcWarps, NS = kTcStages;
   constexpr int smem = tc_dynamic_smem<D, NW, NS>();
   static std::atomic<uint64_t> attr_done{0};
-  auto kern = decode_tc_bf16<D, NT, NW, NS>;
+  auto kern = decode_tc_bf16<D, NT, NW, NS, MODE>;
   if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
   CUtensorMap kmap, vmap;
   if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
-  kern<<<grid, NW * 32, smem, st>>>(kmap, vmap, a);
-  return after_launch();
-}
-
-// Persistent fused kernel: as many CTAs as fit on the GPU at once (at most
-// kMaxStreamWarps warps in all, which bounds the piece storage).
-constexpr int kMaxStreamWarps = 2048;
-
-int sm_count() {
-  static std::atomic<int> cached[kMaxDevices];
-  const int dev = current_device();
-  if (dev < 0 || dev >= kMaxDevices) return -1;
-  int n = cached[dev].load(std::memory_order_relaxed);
-  if (n > 0) return n;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-  cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
-
-template <int D, int NT>
-int launch_tc_streamk(const DecodeArgs& a, const PieceStore& ps, cudaStream_t st) {
-  constexpr int NW = kTcWarps, NS = kTcStages;
-  constexpr int smem = tc_dynamic_smem<D, NW, NS>();
-  static std::atomic<uint64_t> attr_done{0};
-  static std::atomic<int> per_sm[kMaxDevices];
-  auto kern = decode_tc_bf16_streamk<D, NT, NW, NS>;
-  if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
-  const int dev = current_device();
-  const int sms = sm_count();
-  if (dev < 0 || sms <= 0) return GQA_ERR_CUDA;
-  int occ = per_sm[dev].load(std::memory_order_relaxed);
-  if (occ <= 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NW * 32, smem) != cudaSuccess ||
-        occ <= 0)
-      return GQA_ERR_CUDA;
-    per_sm[dev].store(occ, std::memory_order_relaxed);
-  }
-  int ctas = sms * occ;
-  if (ctas * NW > kMaxStreamWarps) ctas = kMaxStreamWarps / NW;
-  CUtensorMap kmap, vmap;
-  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
-    return GQA_ERR_CUDA;
-  kern<<<ctas, NW * 32, smem, st>>>(kmap, vmap, a, ps);
-  return after_launch();
+  return launch_pdl(kern, grid, dim3(NW * 32), smem, st, kmap, vmap, a);
 }
 
 template <int D, int HB, int MODE>
 int launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   constexpr int NW = 4;
-  decode_simt_f32<D, HB, NW, MODE><<<grid, NW * 32, 0, st>>>(a);
-  return after_launch();
+  return launch_pdl(decode_simt_f32<D, HB, NW, MODE>, grid, dim3(NW * 32), 0, st, a);
 }
 
 template <int D, int MODE>
@@ -192,29 +171,20 @@ int launch_simt_hb(const DecodeArgs& a, int hb, dim3 grid, cudaStream_t st) {
   }
 }
 
-// bf16 partials or any fp32 work: one CTA per (split, kv head, head block, b).
+// One CTA per (split, kv head, head block, b).
 template <int MODE>
-int launch_per_split(DecodeArgs a, int dtype, int D, cudaStream_t st) {
+int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
   const int hb = heads_per_cta(dtype, a.G);
   a.n_hb = (a.G + hb - 1) / hb;
   const dim3 grid(a.n_slots, a.h_kv * a.n_hb, a.B);
   if (dtype == GQA_BF16) {
     const bool wide = hb == 16;
-    if (D == 128) return wide ? launch_tc<128, 2>(a, grid, st) : launch_tc<128, 1>(a, grid, st);
-    return wide ? launch_tc<64, 2>(a, grid, st) : launch_tc<64, 1>(a, grid, st);
+    if (D == 128)
+      return wide ? launch_tc<128, 2, MODE>(a, grid, st) : launch_tc<128, 1, MODE>(a, grid, st);
+    return wide ? launch_tc<64, 2, MODE>(a, grid, st) : launch_tc<64, 1, MODE>(a, grid, st);
   }
   if (D == 128) return launch_simt_hb<128, MODE>(a, hb, grid, st);
   return launch_simt_hb<64, MODE>(a, hb, grid, st);
-}
-
-// Fused bf16: the persistent even-split kernel.
-int launch_fused_bf16(DecodeArgs a, const PieceStore& ps, int D, cudaStream_t st) {
-  const int hb = tc_heads_per_cta(a.G);
-  a.n_hb = (a.G + hb - 1) / hb;
-  const bool wide = hb == 16;
-  if (D == 128)
-    return wide ? launch_tc_streamk<128, 2>(a, ps, st) : launch_tc_streamk<128, 1>(a, ps, st);
-  return wide ? launch_tc_streamk<64, 2>(a, ps, st) : launch_tc_streamk<64, 1>(a, ps, st);
 }
 
 // ------------------------------------------------------------ validation
@@ -300,8 +270,7 @@ size_t n_tickets(const Shape& s) {
   return (size_t)s.B * s.h_kv * (G <= 16 ? 1 : (G + 15) / 16);
 }
 
-// fp32 fused path: one triplet per (b, h, split).
-WsLayout ws_layout_triplets(const Shape& s) {
+WsLayout ws_layout(const Shape& s) {
   const size_t rows = (size_t)s.B * s.h_q;
   WsLayout w;
   w.tickets = 0;
@@ -310,47 +279,6 @@ WsLayout ws_layout_triplets(const Shape& s) {
   w.o = w.l + round_up(rows * s.n_slots * sizeof(float), 256);
   w.total = w.o + round_up(rows * s.n_slots * s.D * sizeof(float), 256);
   return w;
-}
-
-// bf16 fused path: pieces, one per (unit, run) pair that meet; at most
-// (non-empty units) + max(warps, kv heads x head blocks) of them, each
-// holding min(16, G) heads.
-int piece_heads(const Shape& s) {
-  const int G = s.h_q / s.h_kv;
-  const int hb = tc_heads_per_cta(G);
-  return G < hb ? G : hb;
-}
-
-size_t piece_slots(const Shape& s) {
-  const int G = s.h_q / s.h_kv;
-  const int hb = tc_heads_per_cta(G);
-  const size_t heads = (size_t)s.h_kv * ((G + hb - 1) / hb);
-  const size_t units = (size_t)s.B * heads * s.n_slots;
-  return units + (heads > (size_t)kMaxStreamWarps ? heads : (size_t)kMaxStreamWarps);
-}
-
-WsLayout ws_layout_pieces(const Shape& s) {
-  const size_t cells = piece_slots(s) * piece_heads(s);
-  WsLayout w;
-  w.tickets = 0;
-  w.m = kTicketBytes;
-  w.l = w.m + round_up(cells * sizeof(float), 256);
-  w.o = w.l + round_up(cells * sizeof(float), 256);
-  w.total = w.o + round_up(cells * s.D * sizeof(float), 256);
-  return w;
-}
-
-WsLayout ws_layout(const Shape& s) {
-  return s.dtype == GQA_BF16 ? ws_layout_pieces(s) : ws_layout_triplets(s);
-}
-
-// Bytes that serve either dtype (the size queries take no dtype).
-size_t ws_bytes_any_dtype(Shape s) {
-  s.dtype = GQA_BF16;
-  const size_t a = ws_layout(s).total;
-  s.dtype = GQA_F32;
-  const size_t b = ws_layout(s).total;
-  return a > b ? a : b;
 }
 
 struct LibWorkspace {
@@ -403,19 +331,11 @@ int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, f
   DecodeArgs a = make_args(q, k, v, seqlens, s);
   uint8_t* base = static_cast<uint8_t*>(ws);
   a.tickets = reinterpret_cast<int*>(base + w.tickets);
-  a.out = out;
-  if (s.dtype == GQA_BF16) {
-    PieceStore ps;
-    ps.m = reinterpret_cast<float*>(base + w.m);
-    ps.l = reinterpret_cast<float*>(base + w.l);
-    ps.o = reinterpret_cast<float*>(base + w.o);
-    ps.HBs = piece_heads(s);
-    return launch_fused_bf16(a, ps, s.D, as_stream(stream));
-  }
   a.m = reinterpret_cast<float*>(base + w.m);
   a.l = reinterpret_cast<float*>(base + w.l);
   a.o = reinterpret_cast<float*>(base + w.o);
-  return launch_per_split<kFused>(a, s.dtype, s.D, as_stream(stream));
+  a.out = out;
+  return launch_decode<kFused>(a, s.dtype, s.D, as_stream(stream));
 }
 
 int partial(const void* q, const void* k, const void* v, const int32_t* seqlens, float* m,
@@ -428,7 +348,7 @@ int partial(const void* q, const void* k, const void* v, const int32_t* seqlens,
   a.m = m;
   a.l = l;
   a.o = o;
-  return launch_per_split<kPartial>(a, s.dtype, s.D, as_stream(stream));
+  return launch_decode<kPartial>(a, s.dtype, s.D, as_stream(stream));
 }
 
 __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
@@ -467,14 +387,14 @@ const char* gqa_decode_error_string(int status) {
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits) {
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, 1.f, GQA_BF16);
   if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
-  return ws_bytes_any_dtype(s);
+  return ws_layout(s).total;
 }
 
 size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head, int chunk_len,
                                          int max_seqlen) {
   const Shape s = chunk_shape(B, h_q, h_kv, d_head, chunk_len, max_seqlen, 1.f, GQA_BF16);
   if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
-  return ws_bytes_any_dtype(s);
+  return ws_layout(s).total;
 }
 
 int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
@@ -520,12 +440,10 @@ int mlo_merge(const float* m, const float* l, const float* o, float* out, int ro
   const dim3 grid((rows + 3) / 4);
   cudaStream_t st = as_stream(stream);
   if (d_head <= 64)
-    mlo_merge_kernel<2><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
-  else if (d_head <= 128)
-    mlo_merge_kernel<4><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
-  else
-    mlo_merge_kernel<8><<<grid, 128, 0, st>>>(m, l, o, out, rows, n_splits, d_head);
-  return after_launch();
+    return launch_pdl(mlo_merge_kernel<2>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
+  if (d_head <= 128)
+    return launch_pdl(mlo_merge_kernel<4>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
+  return launch_pdl(mlo_merge_kernel<8>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
 }
 
 int gqa_decode_get_status(void* stream) {

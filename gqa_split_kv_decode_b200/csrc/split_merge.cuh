@@ -135,10 +135,13 @@ __device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const f
 // Merges n triplets of one row and normalises: the whole warp cooperates,
 // lane j owning elements j, j+32, ... (d <= 32*MAXK).  Splits are combined
 // strictly in index order, so every element's result is deterministic and
-// identical wherever this function runs.  m in natural-log units.
+// identical wherever this function runs.  m in natural-log units.  The o rows
+// of 8 splits are loaded before any of them is used, so a merge costs a few
+// memory round trips rather than one per split.
 template <int MAXK>
 __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
                                                int n, int d, float* out, int lane) {
+  constexpr int BATCH = 8;
   float M = -INFINITY;
   for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(m + i));
   M = warp_max(M);
@@ -155,15 +158,27 @@ __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, c
         li = __ldcg(l + i);
       }
       const int cnt = min(32, n - base);
-      for (int j = 0; j < cnt; ++j) {
-        const float wj = __shfl_sync(kFull, wi, j);
-        const float lj = __shfl_sync(kFull, li, j);
-        L = fmaf(lj, wj, L);
-        const float* oj = o + (size_t)(base + j) * d;
+      for (int j0 = 0; j0 < cnt; j0 += BATCH) {
+        float ov[BATCH][MAXK];
 #pragma unroll
-        for (int k = 0; k < MAXK; ++k) {
-          const int dd = lane + 32 * k;
-          if (dd < d) acc[k] = fmaf(__ldcg(oj + dd), wj, acc[k]);
+        for (int u = 0; u < BATCH; ++u) {
+          const float* oj = o + (size_t)(base + j0 + u) * d;
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int dd = lane + 32 * k;
+            ov[u][k] = (j0 + u < cnt && dd < d) ? __ldcg(oj + dd) : 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+          const int j = j0 + u;
+          const float wj = __shfl_sync(kFull, wi, j & 31);
+          const float lj = __shfl_sync(kFull, li, j & 31);
+          if (j < cnt) {
+            L = fmaf(lj, wj, L);
+#pragma unroll
+            for (int k = 0; k < MAXK; ++k) acc[k] = fmaf(ov[u][k], wj, acc[k]);
+          }
         }
       }
     }
@@ -212,6 +227,8 @@ __global__ void __launch_bounds__(128) mlo_merge_kernel(const float* __restrict_
                                                         const float* __restrict__ o,
                                                         float* __restrict__ out, int rows, int n,
                                                         int d) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
   merge_row_warp<MAXK>(m + (size_t)row * n, l + (size_t)row * n, o + (size_t)row * n * d, n, d,

@@ -104,24 +104,17 @@ def test_partial_and_merge_argument_checks(lib):
 
 
 def test_workspace_size_arithmetic(lib):
-    """Fixed 256 KiB ticket area, then the larger of the two fused layouts:
-    fp32 triplets (m, l, o for every (b, h, split)) or bf16 pieces (one per
-    (unit, warp) pair that meet: at most units + 2048, min(16, G) heads each)."""
+    """Fixed 256 KiB ticket area, then fp32 triplets: m, l [B*h_q][n] and
+    o [B*h_q][n][d], each 256-byte rounded."""
     r = lambda x: (x + 255) // 256 * 256
     T = 256 * 1024
 
-    def expect(B, hq, hkv, d, n):
-        G = hq // hkv
-        trip = 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
-        blocks = 1 if G <= 16 else -(-G // 16)
-        cells = (B * hkv * blocks * n + 2048) * min(G, 8 if G <= 8 else 16)
-        pieces = 2 * r(cells * 4) + r(cells * d * 4)
-        return T + max(trip, pieces)
+    def expect(B, hq, d, n):
+        return T + 2 * r(B * hq * n * 4) + r(B * hq * n * d * 4)
 
-    assert lib.gqa_decode_workspace_size(8, 64, 8, 128, 8) == expect(8, 64, 8, 128, 8)
-    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == expect(1, 32, 1, 128, 2)
-    assert lib.gqa_decode_workspace_size(64, 32, 8, 128, 3) == expect(64, 32, 8, 128, 3)
-    assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == expect(64, 32, 8, 128, 32)
+    assert lib.gqa_decode_workspace_size(8, 64, 8, 128, 8) == expect(8, 64, 128, 8)
+    assert lib.gqa_decode_workspace_size(1, 32, 1, 128, 2) == expect(1, 32, 128, 2)
+    assert lib.gqa_decode_chunked_workspace_size(64, 32, 8, 128, 1024, 32768) == expect(64, 32, 128, 32)
     assert lib.gqa_decode_workspace_size(1, 6, 4, 128, 4) == 0
     assert lib.gqa_decode_workspace_size(1, 8, 2, 96, 4) == 0
     # more than 65536 tickets (B * h_kv * head blocks) is refused
