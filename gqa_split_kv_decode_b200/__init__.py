@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = [
-    "gqa_decode_attn", "gqa_decode_attn_chunked", "gqa_decode_partial",
+    "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
     "get_status", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
@@ -50,6 +50,8 @@ _ws_size = _sig("gqa_decode_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci)
 _ws_size_chunked = _sig("gqa_decode_chunked_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci, _ci)
 _attn = _sig("gqa_decode_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _ci,
              _vp, _sz, _vp)
+_attn_noalloc = _sig("gqa_decode_attn_noalloc", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
+                     _ci, _cf, _ci, _vp)
 _attn_chunked = _sig("gqa_decode_attn_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
                      _ci, _ci, _cf, _ci, _vp, _sz, _vp)
 _partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
@@ -173,6 +175,24 @@ def gqa_decode_attn(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, out
                      out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                      _stream(q.device)), "gqa_decode_attn")
+    return out
+
+
+def gqa_decode_attn_noalloc(q, k_cache, v_cache, seqlens, n_splits: int, scale=None,
+                            out=None) -> torch.Tensor:
+    """gqa_decode_attn for callers that cannot allocate device memory.
+
+    The scratch is a fixed 40 MiB array inside the library (one per device),
+    so the call itself allocates nothing; shapes that need more scratch raise
+    GQADecodeError (ERR_WORKSPACE).  Calls share that array: keep them on one
+    stream.  (Passing ``out=None`` still lets torch allocate the result here;
+    pass ``out`` to avoid even that.)"""
+    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out(out, (B, h_q, d), q.device)
+    with torch.cuda.device(q.device):
+        _check(_attn_noalloc(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+                             out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
+                             _stream(q.device)), "gqa_decode_attn_noalloc")
     return out
 
 

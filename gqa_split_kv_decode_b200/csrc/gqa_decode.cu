@@ -351,6 +351,39 @@ int partial(const void* q, const void* k, const void* v, const int32_t* seqlens,
   return launch_decode<kPartial>(a, s.dtype, s.D, as_stream(stream));
 }
 
+// ------------------------------------------------ allocation-free variant
+
+// Scratch for gqa_decode_attn_noalloc: a fixed array in this module's global
+// memory, so that entry point never allocates.  Every device that loads the
+// library holds these bytes until the process exits.  The first 256 KiB are
+// the ticket area, the rest holds the triplets, exactly as in a caller's
+// workspace.
+constexpr size_t kNoAllocScratchBytes = 40ull << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array, looked up once per device.  In host
+// code `g_noalloc_scratch` only names a host-side stand-in; handing that name
+// to a kernel would read the wrong memory, so the address always comes from
+// cudaGetSymbolAddress with the device current.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];
+
+int noalloc_scratch(void** out) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GQA_OK;
+}
+
 __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -404,6 +437,26 @@ int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
   return fused(q, k_cache, v_cache, seqlens, out,
                split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype), workspace,
                workspace_bytes, stream);
+}
+
+int gqa_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* seqlens, float* out, int B, int h_q, int h_kv,
+                            int d_head, int n_splits, float scale, int dtype, void* stream) {
+  const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype);
+  if (int rc = check_common(q, k_cache, v_cache, seqlens, s)) return rc;
+  if (n_tickets(s) * sizeof(int) > kTicketBytes) return GQA_ERR_UNSUPPORTED;
+  if (s.B == 0) return GQA_OK;
+  const size_t need = ws_layout(s).total;
+  if (need > kNoAllocScratchBytes) return GQA_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  // The array keeps whatever the previous call left; the tickets must start
+  // at zero, so clear this call's part of the ticket area first.
+  if (cudaMemsetAsync(scratch, 0, n_tickets(s) * sizeof(int), as_stream(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  return fused(q, k_cache, v_cache, seqlens, out, s, scratch, kNoAllocScratchBytes, stream);
 }
 
 int gqa_decode_attn_chunked(const void* q, const void* k_cache, const void* v_cache,

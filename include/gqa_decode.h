@@ -122,6 +122,32 @@ GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_ca
                     int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * gqa_decode_attn without any allocation.  No passage of the method's pages
+ * corresponds to this entry point; it exists for callers that cannot call
+ * cudaMalloc -- for example a plugin inside a host program that owns every
+ * device allocation through its own pool, or a latency-critical path that
+ * cannot afford the device-wide synchronisation cudaMalloc may imply.
+ *
+ * Same arguments and result as gqa_decode_attn minus the workspace: the
+ * scratch (ticket area + triplets) is a fixed 40 MiB array in the library's
+ * own device memory, held by every device that loads the library until the
+ * process exits.  A call whose scratch would exceed 40 MiB
+ * (gqa_decode_workspace_size(...) > 40 MiB) returns GQA_ERR_WORKSPACE and
+ * launches nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call clears the tickets it uses
+ * (cudaMemsetAsync on the stream) and then runs the fused kernel; nothing is
+ * allocated or freed.  All calls on a device share that device's one array,
+ * which keeps the last call's contents: calls that overlap on the GPU (for
+ * instance on two streams) race and corrupt each other's results, so order
+ * them on one stream.
+ */
+GQA_API int gqa_decode_attn_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *seqlens, float *out,
+                                    int B, int h_q, int h_kv, int d_head, int n_splits,
+                                    float scale, int dtype, void *stream);
+
+/*
  * Fused decode attention with fixed-length chunks (ragged batches): split i
  * of sequence b covers [i*chunk_len, min((i+1)*chunk_len, S_b)); the last
  * chunk may be partial.  max_seqlen bounds every S_b (host-known, so no
