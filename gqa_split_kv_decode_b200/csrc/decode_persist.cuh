@@ -1,0 +1,362 @@
+// Fused bf16 decode: persistent CTAs over the non-empty splits, then a merge
+// kernel over all rows.
+//
+// The per-split grid runs one CTA per (split, kv head, head block, b); when
+// there are more splits than resident CTAs the second wave starts cold and
+// every wave pays its start-up and drain with the memory system idle.  Here
+// the grid is exactly the CTAs that fit at once, and CTA c takes the
+// non-empty splits ("units") c, c + C, c + 2C, ... in the per-split grid's
+// order (split fastest, then kv head / head block, then b), so CTAs that run
+// together still read neighbouring cache rows.  Each warp keeps one TMA ring
+// across its CTA's units: while the warps of a CTA reduce one split, the
+// first tiles of their next split are already in flight.
+//
+// Per unit, the warps' partial triplets are combined pairwise through an
+// 8 KiB exchange buffer (named barriers), and warp 0 stores the split's
+// triplet (kernbench "_attention_mesh_mlo.py": "One-shot local partial
+// attention").  merge_rows_kernel then merges each row's non-empty splits
+// with the page's log-sum-exp rule and normalises ("Final normalize").
+#pragma once
+
+#include "decode_tc.cuh"
+
+namespace gqa {
+
+// Geometry of one unit (non-empty split of one (b, kv head / head block)).
+struct Unit {
+  int b, gy, slot;
+  int lo, hi;      // keys [lo, hi) of the split, relative to the sequence
+  int ntiles;      // 16-key tiles of the split
+  long long off;   // packed row of the sequence's first key
+};
+
+// Non-empty splits of a sequence: ceil(S / L), clipped to n_slots (0 when
+// S <= 0).  L as in locate_split.
+__device__ __forceinline__ int active_splits(const DecodeArgs& a, int S, long long& L) {
+  if (S <= 0) {
+    L = 1;
+    return 0;
+  }
+  L = a.n_splits > 0 ? ((long long)S + a.n_splits - 1) / a.n_splits : (long long)a.chunk_len;
+  long long n = ((long long)S + L - 1) / L;
+  return (int)(n < a.n_slots ? n : a.n_slots);
+}
+
+__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long x = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += x;
+  }
+  return v;
+}
+
+// Total number of units (whole warp).
+__device__ long long count_units(const DecodeArgs& a, int H, int lane) {
+  long long total = 0;
+  for (int base = 0; base < a.B; base += 32) {
+    const int b = base + lane;
+    long long L;
+    const int n = b < a.B ? active_splits(a, __ldg(a.seqlens + b), L) : 0;
+    total += __shfl_sync(kFull, warp_incl_scan((long long)H * n, lane), 31);
+  }
+  return total;
+}
+
+// Unit u, 0 <= u < count_units (whole warp): scan the sequences for the one
+// holding u, then split u's remainder into (kv head / head block, split).
+__device__ Unit unit_at(const DecodeArgs& a, int H, long long u, int lane) {
+  long long units = 0, rows = 0;
+  for (int base = 0; base < a.B; base += 32) {
+    const int b = base + lane;
+    const int S = b < a.B ? __ldg(a.seqlens + b) : 0;
+    long long L;
+    const int n = b < a.B ? active_splits(a, S, L) : 0;
+    const long long cu = (long long)H * n, cr = S > 0 ? S : 0;
+    const long long iu = warp_incl_scan(cu, lane), ir = warp_incl_scan(cr, lane);
+    const unsigned hit = __ballot_sync(kFull, units + iu > u);
+    if (hit) {
+      const int j = __ffs(hit) - 1;
+      Unit x;
+      x.b = base + j;
+      const long long r = u - (units + __shfl_sync(kFull, iu - cu, j));
+      x.off = rows + __shfl_sync(kFull, ir - cr, j);
+      const int Sj = __shfl_sync(kFull, S, j);
+      long long Lj;
+      const int nj = active_splits(a, Sj, Lj);
+      x.gy = (int)(r / nj);
+      x.slot = (int)(r - (long long)x.gy * nj);
+      long long lo = (long long)x.slot * Lj, hi = lo + Lj;
+      if (hi > Sj) hi = Sj;
+      x.lo = (int)lo;
+      x.hi = (int)hi;
+      x.ntiles = (int)((hi - lo + kTileKeys - 1) / kTileKeys);
+      return x;
+    }
+    units += __shfl_sync(kFull, iu, 31);
+    rows += __shfl_sync(kFull, ir, 31);
+  }
+  Unit none{};  // not reached for u < count_units
+  return none;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// A warp's partial triplet in the exchange buffer: m and l per head column,
+// then the o fragments stored element-major ([i][lane]) so every store and
+// load of a warp touches 32 consecutive words.
+template <int D, int NT>
+struct XSlot {
+  static constexpr int kFrag = (D / 16) * NT * 4;  // o floats per lane
+  static constexpr int kFloats = 2 * NT * 8 + kFrag * 32;
+};
+
+template <int D, int NT>
+__device__ __forceinline__ void xslot_store(float* x, const WarpAcc<D, NT>& acc, int lane) {
+  if (lane < 4) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        x[nt * 8 + 2 * lane + j] = acc.m[nt][j];
+        x[NT * 8 + nt * 8 + 2 * lane + j] = acc.l[nt][j];
+      }
+  }
+  float* xo = x + 2 * NT * 8;
+  int i = 0;
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e, ++i) xo[i * 32 + lane] = acc.o[dt][nt][e];
+}
+
+// acc <- merge(acc, partial in x) with the log-sum-exp rule (base-2 m).
+template <int D, int NT>
+__device__ __forceinline__ void xslot_merge(WarpAcc<D, NT>& acc, const float* x, int lane) {
+  float sa[NT][2], sb[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int h = nt * 8 + 2 * (lane & 3) + j;
+      const float mb = x[h], lb = x[NT * 8 + h];
+      const float M = fmaxf(acc.m[nt][j], mb);
+      sa[nt][j] = M == -INFINITY ? 0.f : exp2f(acc.m[nt][j] - M);
+      sb[nt][j] = M == -INFINITY ? 0.f : exp2f(mb - M);
+      acc.l[nt][j] = acc.l[nt][j] * sa[nt][j] + lb * sb[nt][j];
+      acc.m[nt][j] = M;
+    }
+  const float* xo = x + 2 * NT * 8;
+  int i = 0;
+#pragma unroll
+  for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e, ++i)
+        acc.o[dt][nt][e] = acc.o[dt][nt][e] * sa[nt][e & 1] + xo[i * 32 + lane] * sb[nt][e & 1];
+}
+
+template <int D, int NT, int NW, int NS>
+constexpr int persist_dynamic_smem() {
+  return NW * NS * TcShape<D>::kStageBytes + 2 * XSlot<D, NT>::kFloats * 4 + 1024;
+}
+
+template <int D, int NT, int NW, int NS>
+__global__ void __launch_bounds__(NW * 32)
+    decode_tc_bf16_persist(const __grid_constant__ CUtensorMap kmap,
+                           const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
+  static_assert(NW == 4, "the pairwise exchange assumes four warps");
+  constexpr int HB = NT * 8;
+  constexpr int STAGE = TcShape<D>::kStageBytes;
+  constexpr int STEPS = TcShape<D>::kSteps;
+  constexpr int HALVES = TcShape<D>::kHalves;
+  constexpr int XF = XSlot<D, NT>::kFloats;
+
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[NW * NS];
+  uint8_t* stages = aligned_dyn_smem(dyn_smem);
+  float* xbuf = reinterpret_cast<float*>(stages + NW * NS * STAGE);  // 2 slots of XF floats
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = a.h_kv * a.n_hb;
+
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+#pragma unroll
+    for (int i = 0; i < NW * NS; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
+    fence_barrier_init();
+  }
+  grid_dependency_wait();
+  allow_dependent_launch();
+  __syncthreads();
+
+  if (blockIdx.x == 0 && threadIdx.x < 32) {  // report bad lengths once
+    for (int b = lane; b < a.B; b += 32) {
+      const int S = __ldg(a.seqlens + b);
+      if (S < 0) raise_status(kStatusNegSeqlen);
+      if (a.chunk_len > 0 && (long long)S > (long long)a.n_slots * a.chunk_len)
+        raise_status(kStatusSeqlenOverMax);
+    }
+  }
+
+  const long long A = count_units(a, H, lane);
+  const uint64_t policy = l2_policy_evict_first();
+  const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
+  const uint32_t bar0 = smem_u32(&full_bar[warp * NS]);
+
+  // ---- issue cursor: the next tile of this warp's sequence (warp-uniform)
+  long long ia = blockIdx.x;
+  Unit iu{};
+  int it = warp;
+  bool more = false;
+  if (ia < A) {
+    iu = unit_at(a, H, ia, lane);
+    more = true;
+    while (more && it >= iu.ntiles) {  // no tile of this unit for this warp
+      ia += gridDim.x;
+      if (ia >= A) {
+        more = false;
+      } else {
+        iu = unit_at(a, H, ia, lane);
+        it = warp;
+      }
+    }
+  }
+  uint32_t issued = 0, used = 0;
+  auto issue_next = [&]() {
+    if (lane == 0) {
+      const int ts = iu.lo + it * kTileKeys;
+      const int row0 = (ts + kTileKeys <= iu.hi) ? ts : iu.hi - kTileKeys;
+      tc_issue_stage<D>(stage0 + (issued % NS) * STAGE, bar0 + (issued % NS) * 8, &kmap, &vmap,
+                        iu.gy / a.n_hb, static_cast<int>(iu.off + row0), policy);
+    }
+    ++issued;
+    it += NW;
+    while (it >= iu.ntiles) {
+      ia += gridDim.x;
+      if (ia >= A) {
+        more = false;
+        break;
+      }
+      iu = unit_at(a, H, ia, lane);
+      it = warp;
+    }
+  };
+  for (int s = 0; s < NS && more; ++s) issue_next();
+  __syncwarp();
+
+  uint32_t qf[NT][STEPS][2];
+  int q_b = -1, q_gy = -1;
+  WarpAcc<D, NT> acc;
+  bool failed = false;
+
+  for (long long u = blockIdx.x; u < A; u += gridDim.x) {
+    const Unit cu = unit_at(a, H, u, lane);
+    const int g = cu.gy / a.n_hb, hb = cu.gy % a.n_hb;
+    if (cu.b != q_b || cu.gy != q_gy) {
+      load_q_frags<D, NT>(qf, a, cu.b, g, hb, lane);
+      q_b = cu.b;
+      q_gy = cu.gy;
+    }
+    acc.reset();
+    for (int t = warp; t < cu.ntiles && !failed; t += NW) {
+      const int s = used % NS;
+      const bool ok = mbar_wait_bounded(bar0 + s * 8, (used / NS) & 1, a.timeout_ns);
+      if (!__all_sync(kFull, ok)) {
+        failed = true;
+        break;
+      }
+      const int ts = cu.lo + t * kTileKeys;
+      const int row0 = (ts + kTileKeys <= cu.hi) ? ts : cu.hi - kTileKeys;
+      const uint32_t kbase = stage0 + s * STAGE;
+      tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
+                     row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
+      ++used;
+      __syncwarp();
+      if (more) {
+        if (lane == 0) fence_proxy_async_smem();
+        issue_next();
+      }
+    }
+    if (failed) {
+      // Record the error, let this warp's issued loads land (bounded); the
+      // warp's partials read as empty from here on.
+      if (lane == 0) raise_status(kStatusTimeout);
+      for (uint32_t i = used; i < issued; ++i)
+        mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
+      used = issued;
+      more = false;
+      acc.reset();
+    }
+    acc.reduce_l();
+
+    // ---- combine the four warps' partials: (2,3) -> (0,1), then 1 -> 0
+    named_barrier(1, NW * 32);  // every warp done with this unit and with xbuf
+    if (warp >= 2) xslot_store<D, NT>(xbuf + (warp - 2) * XF, acc, lane);
+    named_barrier(1, NW * 32);
+    if (warp < 2) {
+      xslot_merge<D, NT>(acc, xbuf + warp * XF, lane);
+      named_barrier(2, 64);
+      if (warp == 1) xslot_store<D, NT>(xbuf, acc, lane);
+      named_barrier(3, 64);
+      if (warp == 0) {
+        xslot_merge<D, NT>(acc, xbuf, lane);
+        // ---- store the split's triplet (m in natural-log units)
+        if (lane < 4) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int gi = hb * HB + nt * 8 + 2 * lane + j;
+              if (gi < a.G) {
+                const size_t r = query_row(a, cu.b, g, gi) * a.n_slots + cu.slot;
+                a.m[r] = acc.m[nt][j] == -INFINITY ? -INFINITY : acc.m[nt][j] * kLn2;
+                a.l[r] = acc.l[nt][j];
+              }
+            }
+        }
+#pragma unroll
+        for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int gi = hb * HB + nt * 8 + 2 * (lane & 3) + (e & 1);
+              if (gi < a.G) {
+                const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
+                a.o[(query_row(a, cu.b, g, gi) * a.n_slots + cu.slot) * D + d] = acc.o[dt][nt][e];
+              }
+            }
+      }
+    }
+  }
+}
+
+// Merge of every row's non-empty splits (fused path): one warp per row;
+// a row of an empty sequence is 0.
+template <int MAXK>
+__global__ void __launch_bounds__(128) merge_rows_kernel(const DecodeArgs a, int D) {
+  grid_dependency_wait();
+  allow_dependent_launch();
+  const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= (long long)a.B * a.h_q) return;
+  const int b = (int)(row / a.h_q);
+  long long L;
+  const int n = active_splits(a, __ldg(a.seqlens + b), L);
+  const int lane = threadIdx.x & 31;
+  float* out = a.out + row * D;
+  if (n == 0) {
+    for (int d = lane; d < D; d += 32) out[d] = 0.f;
+    return;
+  }
+  merge_row_warp<MAXK>(a.m + row * a.n_slots, a.l + row * a.n_slots, a.o + row * a.n_slots * D,
+                       n, D, out, lane);
+}
+
+}  // namespace gqa

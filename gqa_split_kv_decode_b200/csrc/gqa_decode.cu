@@ -15,6 +15,7 @@
 #include <utility>
 
 #include "gqa_decode.h"
+#include "decode_persist.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
 #include "split_merge.cuh"
@@ -154,6 +155,49 @@ int launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   return launch_pdl(kern, grid, dim3(NW * 32), smem, st, kmap, vmap, a);
 }
 
+int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return -1;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Fused bf16: persistent CTAs over the non-empty splits (as many as fit on
+// the GPU at once), then the row merge.  Both launches overlap their
+// predecessor's tail (programmatic dependent launch).
+template <int D, int NT>
+int launch_persist(const DecodeArgs& a, cudaStream_t st) {
+  constexpr int NW = 4, NS = kTcStages;
+  constexpr int smem = persist_dynamic_smem<D, NT, NW, NS>();
+  static std::atomic<uint64_t> attr_done{0};
+  static std::atomic<int> per_sm[kMaxDevices];
+  auto kern = decode_tc_bf16_persist<D, NT, NW, NS>;
+  if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
+  const int dev = current_device();
+  const int sms = sm_count();
+  if (dev < 0 || sms <= 0) return GQA_ERR_CUDA;
+  int occ = per_sm[dev].load(std::memory_order_relaxed);
+  if (occ <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NW * 32, smem) != cudaSuccess ||
+        occ <= 0)
+      return GQA_ERR_CUDA;
+    per_sm[dev].store(occ, std::memory_order_relaxed);
+  }
+  const long long units_max = (long long)a.n_slots * a.h_kv * a.n_hb * a.B;
+  const int ctas = (int)(units_max < (long long)sms * occ ? units_max : (long long)sms * occ);
+  CUtensorMap kmap, vmap;
+  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
+    return GQA_ERR_CUDA;
+  if (int rc = launch_pdl(kern, dim3(ctas), dim3(NW * 32), smem, st, kmap, vmap, a)) return rc;
+  const long long rows = (long long)a.B * a.h_q;
+  return launch_pdl(merge_rows_kernel<D / 32>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st,
+                    a, D);
+}
+
 template <int D, int HB, int MODE>
 int launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   constexpr int NW = 4;
@@ -179,9 +223,13 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
   const dim3 grid(a.n_slots, a.h_kv * a.n_hb, a.B);
   if (dtype == GQA_BF16) {
     const bool wide = hb == 16;
+    if (MODE == kFused) {
+      if (D == 128) return wide ? launch_persist<128, 2>(a, st) : launch_persist<128, 1>(a, st);
+      return wide ? launch_persist<64, 2>(a, st) : launch_persist<64, 1>(a, st);
+    }
     if (D == 128)
-      return wide ? launch_tc<128, 2, MODE>(a, grid, st) : launch_tc<128, 1, MODE>(a, grid, st);
-    return wide ? launch_tc<64, 2, MODE>(a, grid, st) : launch_tc<64, 1, MODE>(a, grid, st);
+      return wide ? launch_tc<128, 2, kPartial>(a, grid, st) : launch_tc<128, 1, kPartial>(a, grid, st);
+    return wide ? launch_tc<64, 2, kPartial>(a, grid, st) : launch_tc<64, 1, kPartial>(a, grid, st);
   }
   if (D == 128) return launch_simt_hb<128, MODE>(a, hb, grid, st);
   return launch_simt_hb<64, MODE>(a, hb, grid, st);
