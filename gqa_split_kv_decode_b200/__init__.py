@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
-    "get_status", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "get_status", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
 
@@ -30,7 +30,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE_TIMEOU
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m gqa_split_kv_decode_b200._build` "
+        f"{LIB_PATH} is missing: build it with `python gqa_split_kv_decode_b200/_build.py` "
         "(nvcc, sm_100a). There is no CPU or eager fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -60,6 +60,7 @@ _partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _
                         _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
 _merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
 _get_status = _sig("gqa_decode_get_status", _ci, _vp)
+_launches = _sig("gqa_decode_launches_per_call", _ci, _ci, _ci, _ci, _ci, _ci, _ci)
 _set_timeout = _sig("gqa_decode_set_wait_timeout_ns", _ci, _ull)
 _selftest = _sig("gqa_decode_selftest_wait_timeout", _ci, _ull, _vp)
 _release = _sig("gqa_decode_release", _ci)
@@ -260,6 +261,16 @@ def mlo_merge(m, l, o, out=None) -> torch.Tensor:
         _check(_merge(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
                       _stream(m.device)), "mlo_merge")
     return out
+
+
+def launches_per_call(B, h_q, h_kv, d, n_slots, dtype=BF16, device=None) -> int:
+    """Kernels one fused call launches for this shape on ``device``."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        n = _launches(B, h_q, h_kv, d, n_slots, dtype)
+    if n < 0:
+        raise GQADecodeError(-n, "gqa_decode_launches_per_call")
+    return n
 
 
 def get_status(device=None) -> int:

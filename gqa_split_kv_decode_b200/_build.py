@@ -1,6 +1,9 @@
 """Builds libgqadecode.so in-tree with nvcc for sm_100a (B200).
 
-    python -m gqa_split_kv_decode_b200._build [--verbose-ptxas]
+    python gqa_split_kv_decode_b200/_build.py [--verbose-ptxas]
+
+Run it as a file (not with -m): importing the package loads the library it
+builds.
 """
 from __future__ import annotations
 

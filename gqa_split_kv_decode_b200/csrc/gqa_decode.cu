@@ -142,9 +142,9 @@ int launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cu
 constexpr int kTcWarps = GQA_TC_WARPS;
 constexpr int kTcStages = GQA_TC_STAGES;
 
-template <int D, int NT, int MODE>
+template <int D, int NT, int MODE, int NS = kTcStages>
 int launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr int NW = kTcWarps, NS = kTcStages;
+  constexpr int NW = kTcWarps;
   constexpr int smem = tc_dynamic_smem<D, NW, NS>();
   static std::atomic<uint64_t> attr_done{0};
   auto kern = decode_tc_bf16<D, NT, NW, NS, MODE>;
@@ -164,6 +164,28 @@ int sm_count() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
   cached[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+// Launch plans of the fused bf16 path, chosen from the grid size alone (the
+// sequence lengths live on the device).  R = CTAs of the per-split kernel
+// (4 warps x 3 stages) that fit on the GPU at once, by shared memory.
+//   units <= R      one wave: per-split grid, in-kernel ticket merge (1 launch)
+//   units <= 4 R    a few waves: persistent CTAs + row merge (2 launches), so
+//                   no later wave starts cold
+//   otherwise       many waves: per-split grid with 2 stages (more CTAs per
+//                   SM), whose tails overlap other CTAs' streaming (1 launch)
+enum FusedPlan { kPlanOneWave = 0, kPlanPersistent = 1, kPlanManyWaves = 2 };
+
+int fused_plan(long long units, int D) {
+  const int sms = sm_count();
+  if (sms <= 0) return -1;
+  const int smem = D == 128 ? tc_dynamic_smem<128, kTcWarps, kTcStages>()
+                            : tc_dynamic_smem<64, kTcWarps, kTcStages>();
+  const long long per_sm = (228 * 1024) / (smem + 1024);  // 1 KiB reserved per CTA
+  const long long R = (long long)sms * (per_sm > 0 ? per_sm : 1);
+  if (units <= R) return kPlanOneWave;
+  if (units <= 4 * R) return kPlanPersistent;
+  return kPlanManyWaves;
 }
 
 // Fused bf16: persistent CTAs over the non-empty splits (as many as fit on
@@ -224,8 +246,23 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
   if (dtype == GQA_BF16) {
     const bool wide = hb == 16;
     if (MODE == kFused) {
-      if (D == 128) return wide ? launch_persist<128, 2>(a, st) : launch_persist<128, 1>(a, st);
-      return wide ? launch_persist<64, 2>(a, st) : launch_persist<64, 1>(a, st);
+      const long long units = (long long)grid.x * grid.y * grid.z;
+      switch (fused_plan(units, D)) {
+        case kPlanOneWave:
+          if (D == 128)
+            return wide ? launch_tc<128, 2, kFused>(a, grid, st) : launch_tc<128, 1, kFused>(a, grid, st);
+          return wide ? launch_tc<64, 2, kFused>(a, grid, st) : launch_tc<64, 1, kFused>(a, grid, st);
+        case kPlanPersistent:
+          if (D == 128) return wide ? launch_persist<128, 2>(a, st) : launch_persist<128, 1>(a, st);
+          return wide ? launch_persist<64, 2>(a, st) : launch_persist<64, 1>(a, st);
+        case kPlanManyWaves:
+          if (D == 128)
+            return wide ? launch_tc<128, 2, kFused, 2>(a, grid, st)
+                        : launch_tc<128, 1, kFused, 2>(a, grid, st);
+          return wide ? launch_tc<64, 2, kFused, 2>(a, grid, st) : launch_tc<64, 1, kFused, 2>(a, grid, st);
+        default:
+          return GQA_ERR_CUDA;
+      }
     }
     if (D == 128)
       return wide ? launch_tc<128, 2, kPartial>(a, grid, st) : launch_tc<128, 1, kPartial>(a, grid, st);
@@ -545,6 +582,19 @@ int mlo_merge(const float* m, const float* l, const float* o, float* out, int ro
   if (d_head <= 128)
     return launch_pdl(mlo_merge_kernel<4>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
   return launch_pdl(mlo_merge_kernel<8>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
+}
+
+int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slots, int dtype) {
+  const Shape s = split_shape(B, h_q, h_kv, d_head, n_slots, 1.f, dtype);
+  if (check_shape(s)) return -GQA_ERR_INVALID_ARG;
+  if (B == 0) return 0;
+  if (dtype != GQA_BF16) return 1;
+  const int G = h_q / h_kv;
+  const int hb = tc_heads_per_cta(G);
+  const long long units = (long long)n_slots * h_kv * ((G + hb - 1) / hb) * B;
+  const int plan = fused_plan(units, d_head);
+  if (plan < 0) return -GQA_ERR_CUDA;
+  return plan == kPlanPersistent ? 2 : 1;
 }
 
 int gqa_decode_get_status(void* stream) {

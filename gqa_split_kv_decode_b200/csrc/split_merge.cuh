@@ -136,39 +136,46 @@ __device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const f
 // lane j owning elements j, j+32, ... (d <= 32*MAXK).  Splits are combined
 // strictly in index order, so every element's result is deterministic and
 // identical wherever this function runs.  m in natural-log units.  The o rows
-// of 8 splits are loaded before any of them is used, so a merge costs a few
-// memory round trips rather than one per split.
+// of the first 8 splits are requested together with m and l, and each later
+// batch of 8 before any of its rows is used, so a merge of up to 8 splits
+// costs about one memory round trip.
 template <int MAXK>
 __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
                                                int n, int d, float* out, int lane) {
   constexpr int BATCH = 8;
-  float M = -INFINITY;
-  for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(m + i));
+  float ov[BATCH][MAXK];
+  auto load_batch = [&](int j0) {  // o rows j0 .. j0 + BATCH - 1 (those < n)
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const float* oj = o + (size_t)(j0 + u) * d;
+#pragma unroll
+      for (int k = 0; k < MAXK; ++k) {
+        const int dd = lane + 32 * k;
+        ov[u][k] = (j0 + u < n && dd < d) ? __ldcg(oj + dd) : 0.f;
+      }
+    }
+  };
+  load_batch(0);  // in flight while the maximum is formed
+  float mi = lane < n ? __ldcg(m + lane) : -INFINITY;
+  float li = lane < n ? __ldcg(l + lane) : 0.f;
+  float M = mi;
+  for (int j = 32 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(m + j));
   M = warp_max(M);
+
   float acc[MAXK];
 #pragma unroll
   for (int k = 0; k < MAXK; ++k) acc[k] = 0.f;
   float L = 0.f;
   if (M != -INFINITY) {
     for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      float wi = 0.f, li = 0.f;
-      if (i < n) {
-        wi = exp2f((__ldcg(m + i) - M) * kLog2e);  // 0 for an empty split
-        li = __ldcg(l + i);
+      if (base > 0) {
+        mi = base + lane < n ? __ldcg(m + base + lane) : -INFINITY;
+        li = base + lane < n ? __ldcg(l + base + lane) : 0.f;
       }
+      const float wi = exp2f((mi - M) * kLog2e);  // 0 for an empty split
       const int cnt = min(32, n - base);
       for (int j0 = 0; j0 < cnt; j0 += BATCH) {
-        float ov[BATCH][MAXK];
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-          const float* oj = o + (size_t)(base + j0 + u) * d;
-#pragma unroll
-          for (int k = 0; k < MAXK; ++k) {
-            const int dd = lane + 32 * k;
-            ov[u][k] = (j0 + u < cnt && dd < d) ? __ldcg(oj + dd) : 0.f;
-          }
-        }
+        if (base + j0 > 0) load_batch(base + j0);
 #pragma unroll
         for (int u = 0; u < BATCH; ++u) {
           const int j = j0 + u;

@@ -191,6 +191,16 @@ GQA_API int mlo_merge(const float *m, const float *l, const float *o, float *out
               int rows, int n_splits, int d_head, void *stream);
 
 /*
+ * Number of kernels one fused call (gqa_decode_attn / _chunked / _noalloc)
+ * launches on the current device for this shape (n_slots = n_splits, or
+ * ceil(max_seqlen / chunk_len) when chunked): 1, or 2 when the persistent
+ * decode kernel plus its row merge is chosen.  0 for B == 0; a negative
+ * gqa_status on bad arguments.
+ */
+GQA_API int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slots,
+                                         int dtype);
+
+/*
  * Synchronises `stream`, then reads and clears this device's status word.
  * Returns GQA_OK, GQA_ERR_DEVICE_TIMEOUT, GQA_ERR_DEVICE_SEQLEN or
  * GQA_ERR_CUDA.

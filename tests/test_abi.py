@@ -6,7 +6,7 @@ import re
 
 import pytest
 
-from gqa_split_kv_decode_b200 import _build
+import importlib.util
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "gqa_decode.h")
@@ -14,9 +14,17 @@ HEADER = os.path.join(ROOT, "include", "gqa_decode.h")
 OK, INVALID, UNSUPPORTED, CUDA_ERR, WORKSPACE = 0, 1, 2, 3, 4
 
 
+def _builder():
+    path = os.path.join(ROOT, "gqa_split_kv_decode_b200", "_build.py")
+    spec = importlib.util.spec_from_file_location("gqa_decode_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 @pytest.fixture(scope="module")
 def lib():
-    path = _build.build()
+    path = _builder().build()
     lib = ctypes.CDLL(path)
     vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.gqa_decode_attn.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
