@@ -41,7 +41,7 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20
 ROTATE_TOTAL = 1 << 30
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_tc_bf16_llama70b.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_tc_bf16_persist_llama70b.md")
 
 
 def parse_args(argv=None):
@@ -355,7 +355,8 @@ def run_ours(args, rank, world, local_rank):
             "kernel": ("decode_tc_bf16_persist + merge_rows_kernel" if launches == 2 else "decode_tc_bf16 (fused)")
                       if cfg.dtype == "bf16" else "decode_simt_f32",
             "launches_per_step": launches,
-            "timing": "CUDA events around the K back-to-back launches of the timed region",
+            "timing": "CUDA events around the K back-to-back steps of the timed region (a step's launches "
+                      "together, so the dominant kernel's own rate is at least this)",
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(max_iso_ms, 6),
         },
