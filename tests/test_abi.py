@@ -127,3 +127,10 @@ def test_workspace_size_arithmetic(lib):
     assert lib.gqa_decode_workspace_size(1, 8, 2, 96, 4) == 0
     # more than 65536 tickets (B * h_kv * head blocks) is refused
     assert lib.gqa_decode_workspace_size(65535, 8, 2, 128, 1) == 0
+
+
+def test_launch_count_query_without_a_gpu(lib):
+    lib.gqa_decode_launches_per_call.argtypes = [ctypes.c_int] * 6
+    assert lib.gqa_decode_launches_per_call(0, 8, 2, 128, 4, 1) == 0      # empty batch
+    assert lib.gqa_decode_launches_per_call(2, 8, 2, 128, 4, 0) == 1      # fp32: one kernel
+    assert lib.gqa_decode_launches_per_call(2, 6, 4, 128, 4, 1) == -INVALID

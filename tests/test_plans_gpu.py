@@ -1,0 +1,90 @@
+"""Each launch plan of the fused bf16 path against the oracle.
+
+The plan follows from the grid size (units = splits x kv heads x head blocks
+x batch) against R, the per-split CTAs resident at once (2 per SM at d = 128,
+4 at d = 64): one wave (units <= R), persistent (R < units <= 4R), many waves
+(units > 4R).  The shapes below land in each plan on a 148-SM B200.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import random_case
+
+pytestmark = pytest.mark.gpu
+
+TOL = (2e-3, 1e-2)
+
+
+@pytest.fixture(scope="module")
+def gk():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import gqa_split_kv_decode_b200 as gk
+    return gk
+
+
+def _check(got, w):
+    c = w.cfg
+    ref = oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale).reshape(c.B, c.h_q, c.d)
+    got = got.double().cpu().numpy()
+    err = np.abs(got - ref)
+    bound = TOL[0] + TOL[1] * np.abs(ref)
+    assert (err <= bound).all(), float((err - bound).max())
+
+
+# (B, h_q, h_kv, d, seqlens, n_splits, launches expected on 148 SMs)
+CASES = [
+    (3, 16, 2, 128, [100, 0, 2000], 4, 1),                   # one wave
+    (4, 64, 8, 128, [0, 1, 17, 3000], 16, 2),                 # persistent; empty and 1-key sequences
+    (4, 64, 4, 128, [900, 2, 0, 4000], 32, 2),                # persistent, 16-head blocks
+    (6, 64, 8, 64, [300, 40, 5000, 1, 77, 1200], 16, 2),      # persistent, d = 64 (R = 4 per SM)
+    (6, 64, 8, 128, [5, 0, 700, 33, 4096, 16], 32, 1),        # many waves
+    (2, 96, 2, 128, [2500, 300], 200, 1),                     # many waves, 3 head blocks of 16
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}_hq{c[1]}_hkv{c[2]}_d{c[3]}_n{c[5]}" for c in CASES])
+def test_plan_matches_oracle(gk, case):
+    B, hq, hkv, d, seqlens, n, launches = case
+    w = random_case(B, hq, hkv, d, seqlens, dtype="bf16", seed=sum(seqlens) % 997)
+    c = w.cfg
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert gk.launches_per_call(B, hq, hkv, d, n) == launches
+    q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
+    for _ in range(2):  # twice: the second call reuses the workspace
+        out = gk.gqa_decode_attn(q, k, v, sl, n, c.scale)
+        torch.cuda.synchronize()
+        assert gk.get_status() == 0
+        _check(out, w)
+
+
+def test_persistent_chunked_ragged(gk):
+    """Chunked policy in the persistent plan: 16 sequences, chunk 64."""
+    rng = np.random.default_rng(5)
+    seqlens = [int(x) for x in rng.integers(0, 300, size=16)]
+    seqlens[3] = 0
+    w = random_case(16, 32, 8, 128, seqlens, dtype="bf16", seed=6)
+    c = w.cfg
+    n_slots = -(-max(seqlens) // 64)
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert gk.launches_per_call(16, 32, 8, 128, n_slots) == 2
+    q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
+    out = gk.gqa_decode_attn_chunked(q, k, v, sl, 64, max(seqlens), c.scale)
+    torch.cuda.synchronize()
+    assert gk.get_status() == 0
+    _check(out, w)
+
+
+def test_persistent_reports_bad_lengths(gk):
+    w = random_case(4, 64, 8, 128, [100, 200, 300, 400], dtype="bf16", seed=7)
+    q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
+    sl[1] = -3
+    out = gk.gqa_decode_attn(q, k, v, sl, 16, w.cfg.scale)
+    assert gk.get_status() == gk.ERR_DEVICE_SEQLEN
+    assert torch.all(out[1] == 0)
+    assert gk.get_status() == 0
+    sl[1] = 200
+    out = gk.gqa_decode_attn_chunked(q, k, v, sl, 16, 256, w.cfg.scale)  # 400 > 256
+    assert gk.get_status() == gk.ERR_DEVICE_SEQLEN
