@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = [
-    "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_chunked", "gqa_decode_partial",
+    "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
     "get_status", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
@@ -52,6 +52,8 @@ _attn = _sig("gqa_decode_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci
              _vp, _sz, _vp)
 _attn_noalloc = _sig("gqa_decode_attn_noalloc", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
                      _ci, _cf, _ci, _vp)
+_attn_append = _sig("gqa_decode_attn_append", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci,
+                    _ci, _ci, _ci, _ci, _cf, _ci, _vp, _sz, _vp)
 _attn_chunked = _sig("gqa_decode_attn_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
                      _ci, _ci, _cf, _ci, _vp, _sz, _vp)
 _partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
@@ -194,6 +196,31 @@ def gqa_decode_attn_noalloc(q, k_cache, v_cache, seqlens, n_splits: int, scale=N
         _check(_attn_noalloc(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
                              out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
                              _stream(q.device)), "gqa_decode_attn_noalloc")
+    return out
+
+
+def gqa_decode_attn_append(q, k_new, v_new, k_cache, v_cache, seqlens, n_splits: int, scale=None,
+                           out=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Writes k_new, v_new ([B, h_kv, d]) into the padded cache ([B, cap, h_kv, d])
+    at row seqlens[b] of each sequence and attends over the seqlens[b] + 1
+    keys.  seqlens is left unchanged (advance it for the next step)."""
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache, v_cache must be [B, cap, h_kv, d]")
+    B, cap, h_kv, d = k_cache.shape
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, h_kv, d) or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor [B, h_kv, d] of q's dtype")
+    _, h_q, _, _, dt = _inputs(q, k_cache.view(B * cap, h_kv, d), v_cache.view(B * cap, h_kv, d), seqlens)
+    out = _out(out, (B, h_q, d), q.device)
+    need = _ws_size(B, h_q, h_kv, d, n_splits)
+    if workspace is None:
+        workspace = _workspace(q.device, need)
+    with torch.cuda.device(q.device):
+        _check(_attn_append(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
+                            v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h_q, h_kv, d, cap,
+                            n_splits, _default_scale(d, scale), dt, workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream(q.device)),
+               "gqa_decode_attn_append")
     return out
 
 

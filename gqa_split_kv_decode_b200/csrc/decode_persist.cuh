@@ -26,12 +26,14 @@ namespace gqa {
 struct Unit {
   int b, gy, slot;
   int lo, hi;      // keys [lo, hi) of the split, relative to the sequence
-  int ntiles;      // 16-key tiles of the split
-  long long off;   // packed row of the sequence's first key
+  int cached_hi;   // min(hi, cached keys): the split's keys read from the cache
+  bool has_new;    // the split holds the appended token (key number cached_hi)
+  int ntiles;      // 16-key tiles of [lo, cached_hi)
+  long long off;   // cache row of the sequence's first key
 };
 
-// Non-empty splits of a sequence: ceil(S / L), clipped to n_slots (0 when
-// S <= 0).  L as in locate_split.
+// Non-empty splits of a sequence attending S keys: ceil(S / L), clipped to
+// n_slots (0 when S == 0).  L as in locate_split.
 __device__ __forceinline__ int active_splits(const DecodeArgs& a, int S, long long& L) {
   if (S <= 0) {
     L = 1;
@@ -57,7 +59,7 @@ __device__ long long count_units(const DecodeArgs& a, int H, int lane) {
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
     long long L;
-    const int n = b < a.B ? active_splits(a, __ldg(a.seqlens + b), L) : 0;
+    const int n = b < a.B ? active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L) : 0;
     total += __shfl_sync(kFull, warp_incl_scan((long long)H * n, lane), 31);
   }
   return total;
@@ -69,10 +71,10 @@ __device__ Unit unit_at(const DecodeArgs& a, int H, long long u, int lane) {
   long long units = 0, rows = 0;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const int S = b < a.B ? __ldg(a.seqlens + b) : 0;
+    const SeqKeys kk = seq_keys(a, b < a.B ? __ldg(a.seqlens + b) : 0);
     long long L;
-    const int n = b < a.B ? active_splits(a, S, L) : 0;
-    const long long cu = (long long)H * n, cr = S > 0 ? S : 0;
+    const int n = b < a.B ? active_splits(a, kk.total, L) : 0;
+    const long long cu = (long long)H * n, cr = kk.cached;
     const long long iu = warp_incl_scan(cu, lane), ir = warp_incl_scan(cr, lane);
     const unsigned hit = __ballot_sync(kFull, units + iu > u);
     if (hit) {
@@ -80,17 +82,21 @@ __device__ Unit unit_at(const DecodeArgs& a, int H, long long u, int lane) {
       Unit x;
       x.b = base + j;
       const long long r = u - (units + __shfl_sync(kFull, iu - cu, j));
-      x.off = rows + __shfl_sync(kFull, ir - cr, j);
-      const int Sj = __shfl_sync(kFull, S, j);
+      x.off = a.cap > 0 ? (long long)x.b * a.cap : rows + __shfl_sync(kFull, ir - cr, j);
+      const int St = __shfl_sync(kFull, kk.total, j), Sc = __shfl_sync(kFull, kk.cached, j);
+      const bool app = __shfl_sync(kFull, kk.append, j);
       long long Lj;
-      const int nj = active_splits(a, Sj, Lj);
+      const int nj = active_splits(a, St, Lj);
       x.gy = (int)(r / nj);
       x.slot = (int)(r - (long long)x.gy * nj);
       long long lo = (long long)x.slot * Lj, hi = lo + Lj;
-      if (hi > Sj) hi = Sj;
+      if (hi > St) hi = St;
       x.lo = (int)lo;
       x.hi = (int)hi;
-      x.ntiles = (int)((hi - lo + kTileKeys - 1) / kTileKeys);
+      x.cached_hi = (int)(hi < Sc ? hi : Sc);
+      x.has_new = app && lo <= Sc && Sc < hi;
+      const long long len = x.cached_hi > x.lo ? x.cached_hi - x.lo : 0;
+      x.ntiles = (int)((len + kTileKeys - 1) / kTileKeys);
       return x;
     }
     units += __shfl_sync(kFull, iu, 31);
@@ -199,8 +205,8 @@ __global__ void __launch_bounds__(NW * 32)
   if (blockIdx.x == 0 && threadIdx.x < 32) {  // report bad lengths once
     for (int b = lane; b < a.B; b += 32) {
       const int S = __ldg(a.seqlens + b);
-      if (S < 0) raise_status(kStatusNegSeqlen);
-      if (a.chunk_len > 0 && (long long)S > (long long)a.n_slots * a.chunk_len)
+      report_length(a, S, true);
+      if (a.chunk_len > 0 && (long long)seq_keys(a, S).total > (long long)a.n_slots * a.chunk_len)
         raise_status(kStatusSeqlenOverMax);
     }
   }
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(NW * 32)
   auto issue_next = [&]() {
     if (lane == 0) {
       const int ts = iu.lo + it * kTileKeys;
-      const int row0 = (ts + kTileKeys <= iu.hi) ? ts : iu.hi - kTileKeys;
+      const int row0 = (ts + kTileKeys <= iu.cached_hi) ? ts : iu.cached_hi - kTileKeys;
       tc_issue_stage<D>(stage0 + (issued % NS) * STAGE, bar0 + (issued % NS) * 8, &kmap, &vmap,
                         iu.gy / a.n_hb, static_cast<int>(iu.off + row0), policy);
     }
@@ -273,8 +279,9 @@ __global__ void __launch_bounds__(NW * 32)
         break;
       }
       const int ts = cu.lo + t * kTileKeys;
-      const int row0 = (ts + kTileKeys <= cu.hi) ? ts : cu.hi - kTileKeys;
+      const int row0 = (ts + kTileKeys <= cu.cached_hi) ? ts : cu.cached_hi - kTileKeys;
       const uint32_t kbase = stage0 + s * STAGE;
+      if (a.cap > 0 && row0 < 0) zero_v_rows<D>(kbase + HALVES * kBoxBytes, -row0, lane);
       tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
                      row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
       ++used;
@@ -293,6 +300,13 @@ __global__ void __launch_bounds__(NW * 32)
       used = issued;
       more = false;
       acc.reset();
+    }
+    if (cu.has_new && warp == cu.ntiles % NW) {  // the appended token, after the cached keys
+      const size_t nr = ((size_t)cu.b * a.h_kv + g) * D;
+      const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + nr;
+      const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + nr;
+      tc_extra_key<D, NT>(acc, qf, kn, vn, a.scale_log2, lane);
+      if (hb == 0) store_new_row<D>(a, kn, vn, cu.off + cu.cached_hi, g, lane);
     }
     acc.reduce_l();
 
@@ -348,7 +362,7 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const DecodeArgs a, int
   if (row >= (long long)a.B * a.h_q) return;
   const int b = (int)(row / a.h_q);
   long long L;
-  const int n = active_splits(a, __ldg(a.seqlens + b), L);
+  const int n = active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L);
   const int lane = threadIdx.x & 31;
   float* out = a.out + row * D;
   if (n == 0) {

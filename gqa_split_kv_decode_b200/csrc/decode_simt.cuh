@@ -53,17 +53,22 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
     for (int e = 0; e < PER; ++e) o_acc[hh][e] = 0.f;
   }
 
+  const size_t new_base = ((size_t)b * a.h_kv + g) * D + lane * PER;
   for (int j = sp.lo + warp; j < sp.hi; j += NW) {
-    const size_t base = ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
+    // key j comes from the cache, or is the appended token (key number cached_hi)
+    const bool fresh = sp.has_new && j == sp.cached_hi;
+    const size_t base = fresh ? new_base : ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
+    const float* ksrc = fresh ? static_cast<const float*>(a.k_new) : kp;
+    const float* vsrc = fresh ? static_cast<const float*>(a.v_new) : vp;
     float kr[PER], vr[PER];
     if constexpr (PER == 4) {
-      const float4 k4 = __ldg(reinterpret_cast<const float4*>(kp + base));
-      const float4 v4 = __ldg(reinterpret_cast<const float4*>(vp + base));
+      const float4 k4 = __ldg(reinterpret_cast<const float4*>(ksrc + base));
+      const float4 v4 = __ldg(reinterpret_cast<const float4*>(vsrc + base));
       kr[0] = k4.x; kr[1] = k4.y; kr[2] = k4.z; kr[3] = k4.w;
       vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
     } else {
-      const float2 k2 = __ldg(reinterpret_cast<const float2*>(kp + base));
-      const float2 v2 = __ldg(reinterpret_cast<const float2*>(vp + base));
+      const float2 k2 = __ldg(reinterpret_cast<const float2*>(ksrc + base));
+      const float2 v2 = __ldg(reinterpret_cast<const float2*>(vsrc + base));
       kr[0] = k2.x; kr[1] = k2.y;
       vr[0] = v2.x; vr[1] = v2.y;
     }
@@ -81,6 +86,15 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
 #pragma unroll
       for (int e = 0; e < PER; ++e) o_acc[hh][e] = fmaf(o_acc[hh][e], alpha, p * vr[e]);
       m_run[hh] = m_new;
+    }
+  }
+
+  if (sp.has_new && hb == 0 && warp == 0) {  // write the appended token's row
+    const size_t dst = ((size_t)(sp.off + sp.cached_hi) * a.h_kv + g) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const_cast<float*>(kp)[dst + e] = static_cast<const float*>(a.k_new)[new_base + e];
+      const_cast<float*>(vp)[dst + e] = static_cast<const float*>(a.v_new)[new_base + e];
     }
   }
 

@@ -199,6 +199,89 @@ __device__ __forceinline__ void tc_tile(WarpAcc<D, NT>& acc, const uint32_t (&qf
   }
 }
 
+// Folds one more key into a warp's online-softmax state: the token being
+// appended, read from global memory (d bf16 values of k and of v for this kv
+// head) rather than from a stage.  Register-only.
+template <int D, int NT>
+__device__ __forceinline__ void tc_extra_key(WarpAcc<D, NT>& acc, const uint32_t (&qf)[NT][D / 16][2],
+                                             const __nv_bfloat16* kn, const __nv_bfloat16* vn,
+                                             float scale_log2, int lane) {
+  constexpr int STEPS = D / 16;
+  const uint32_t* kw = reinterpret_cast<const uint32_t*>(kn);
+  float s_own[NT];  // logit of head 8 nt + lane/4 (the B-fragment head of this lane)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float part = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < STEPS; ++ks) {
+      const uint32_t k0 = __ldg(kw + ks * 8 + (lane & 3));
+      const uint32_t k1 = __ldg(kw + ks * 8 + 4 + (lane & 3));
+      part = fmaf(bf16lo_to_f32(qf[nt][ks][0]), bf16lo_to_f32(k0), part);
+      part = fmaf(bf16hi_to_f32(qf[nt][ks][0]), bf16hi_to_f32(k0), part);
+      part = fmaf(bf16lo_to_f32(qf[nt][ks][1]), bf16lo_to_f32(k1), part);
+      part = fmaf(bf16hi_to_f32(qf[nt][ks][1]), bf16hi_to_f32(k1), part);
+    }
+    part += __shfl_xor_sync(kFull, part, 1);
+    part += __shfl_xor_sync(kFull, part, 2);
+    s_own[nt] = part * scale_log2;
+  }
+  float alpha[NT][2], p[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      // this lane's accumulator column is head 8 nt + 2 (lane%4) + j
+      const float s = __shfl_sync(kFull, s_own[nt], 4 * (2 * (lane & 3) + j));
+      const float mn = fmaxf(acc.m[nt][j], s);
+      alpha[nt][j] = exp2f(acc.m[nt][j] - mn);
+      p[nt][j] = exp2f(s - mn);
+      acc.m[nt][j] = mn;
+      // the 8 lanes of a column each hold part of l: count the new weight once
+      acc.l[nt][j] = acc.l[nt][j] * alpha[nt][j] + ((lane >> 2) == 0 ? p[nt][j] : 0.f);
+    }
+#pragma unroll
+  for (int dt = 0; dt < STEPS; ++dt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
+      const float v = __bfloat162float(vn[d]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        acc.o[dt][nt][e] = fmaf(acc.o[dt][nt][e], alpha[nt][e & 1], p[nt][e & 1] * v);
+    }
+}
+
+// Stores the appended token's k and v rows (d bf16 each) into the cache row
+// `dst_row` of kv head g.  Whole warp.
+template <int D>
+__device__ __forceinline__ void store_new_row(const DecodeArgs& a, const __nv_bfloat16* kn,
+                                              const __nv_bfloat16* vn, long long dst_row, int g,
+                                              int lane) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  const size_t base = ((size_t)dst_row * a.h_kv + g) * D;
+  if (lane < 2 * CH) {
+    const bool isv = lane >= CH;
+    const int c = isv ? lane - CH : lane;
+    const uint4 val = __ldg(reinterpret_cast<const uint4*>(isv ? vn : kn) + c);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(const_cast<void*>(isv ? a.v : a.k)) + base) + c;
+    *dst = val;
+  }
+}
+
+// Zeroes V rows [0, n) of a stage.  In a padded cache the rows before a
+// sequence's first key are the previous sequence's unused tail and may hold
+// anything; masking their weights to 0 would still leave 0 * NaN in P V.
+template <int D>
+__device__ __forceinline__ void zero_v_rows(uint32_t vbase, int n, int lane) {
+  constexpr int CH = (D / 64) * 8;  // 16-byte chunks per row, both d halves
+  for (int c = lane; c < n * CH; c += 32) {
+    const int r = c / CH, rem = c % CH;
+    const uint32_t addr = vbase + (rem >> 3) * kBoxBytes + r * 128 + (rem & 7) * 16;
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+  }
+  __syncwarp();
+}
+
 // Issues the TMA loads of one stage: both d halves of K then of V for the
 // 16 rows starting at packed row `row` of kv head g.
 template <int D>
@@ -264,7 +347,7 @@ __global__ void __launch_bounds__(NW * 32)
     return;
   }
 
-  const int len = sp.hi - sp.lo;
+  const int len = sp.cached_hi > sp.lo ? sp.cached_hi - sp.lo : 0;  // keys read from the cache
   const int ntiles = (len + KT - 1) / KT;
   const uint64_t policy = l2_policy_evict_first();
   const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
@@ -273,7 +356,7 @@ __global__ void __launch_bounds__(NW * 32)
   // First row (relative to the sequence) that tile t loads.
   auto tile_row0 = [&](int t) {
     const int ts = sp.lo + t * KT;
-    return (ts + KT <= sp.hi) ? ts : sp.hi - KT;
+    return (ts + KT <= sp.cached_hi) ? ts : sp.cached_hi - KT;
   };
   auto issue = [&](int t, int s) {
     tc_issue_stage<D>(stage0 + s * STAGE, bar0 + s * 8, &kmap, &vmap, g,
@@ -307,6 +390,7 @@ __global__ void __launch_bounds__(NW * 32)
     const uint32_t kbase = stage0 + s * STAGE;
     const int ts = sp.lo + t * KT;
     const int row0 = tile_row0(t);
+    if (a.cap > 0 && row0 < 0) zero_v_rows<D>(kbase + HALVES * kBoxBytes, -row0, lane);
     tc_tile<D, NT>(acc, qf, kbase, kbase + HALVES * kBoxBytes, row0 + (lane >> 2) >= ts,
                    row0 + (lane >> 2) + 8 >= ts, a.scale_log2, lane);
     __syncwarp();
@@ -326,6 +410,13 @@ __global__ void __launch_bounds__(NW * 32)
     const int last = min(it + NS, my_tiles);
     for (int i = it; i < last; ++i) mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
     acc.reset();
+  }
+  if (sp.has_new && warp == ntiles % NW) {  // the appended token, after the cached keys
+    const size_t nr = ((size_t)b * a.h_kv + g) * D;
+    const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + nr;
+    const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + nr;
+    tc_extra_key<D, NT>(acc, qf, kn, vn, a.scale_log2, lane);
+    if (hb == 0) store_new_row<D>(a, kn, vn, sp.off + sp.cached_hi, g, lane);
   }
   acc.reduce_l();
 

@@ -18,7 +18,7 @@ constexpr unsigned kFull = 0xffffffffu;
 enum : unsigned {
   kStatusTimeout = 1u,        // a bounded wait ran out
   kStatusNegSeqlen = 2u,      // some S_b < 0 (treated as 0)
-  kStatusSeqlenOverMax = 4u,  // chunked mode: S_b > max_seqlen (tail ignored)
+  kStatusSeqlenOverMax = 4u,  // S_b above max_seqlen (chunked) or above a padded cache's room
 };
 
 // Per-device status word of this library (one per loaded module).

@@ -400,8 +400,17 @@ int lib_workspace(size_t need, void** out) {
   return GQA_OK;
 }
 
+// The token to append and the per-sequence capacity of a padded cache
+// ([B][cap][h_kv][d]); all zero for the plain packed-cache calls.
+struct Append {
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  long long cap = 0;
+};
+
 int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, float* out,
-          const Shape& s, void* workspace, size_t workspace_bytes, void* stream) {
+          const Shape& s, void* workspace, size_t workspace_bytes, void* stream,
+          const Append& app = Append()) {
   if (int rc = check_common(q, k, v, seqlens, s)) return rc;
   if (n_tickets(s) * sizeof(int) > kTicketBytes) return GQA_ERR_UNSUPPORTED;
   if (s.B == 0) return GQA_OK;
@@ -414,6 +423,9 @@ int fused(const void* q, const void* k, const void* v, const int32_t* seqlens, f
     return rc;
   }
   DecodeArgs a = make_args(q, k, v, seqlens, s);
+  a.k_new = app.k_new;
+  a.v_new = app.v_new;
+  a.cap = app.cap;
   uint8_t* base = static_cast<uint8_t*>(ws);
   a.tickets = reinterpret_cast<int*>(base + w.tickets);
   a.m = reinterpret_cast<float*>(base + w.m);
@@ -542,6 +554,22 @@ int gqa_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_ca
     return GQA_ERR_CUDA;
   }
   return fused(q, k_cache, v_cache, seqlens, out, s, scratch, kNoAllocScratchBytes, stream);
+}
+
+int gqa_decode_attn_append(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                           void* v_cache, const int32_t* seqlens, float* out, int B, int h_q,
+                           int h_kv, int d_head, int cache_capacity, int n_splits, float scale,
+                           int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype);
+  if (cache_capacity < 1) return GQA_ERR_INVALID_ARG;
+  if ((long long)B * cache_capacity > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;  // int32 rows
+  if (B > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)))
+    return GQA_ERR_INVALID_ARG;
+  Append app;
+  app.k_new = k_new;
+  app.v_new = v_new;
+  app.cap = cache_capacity;
+  return fused(q, k_cache, v_cache, seqlens, out, s, workspace, workspace_bytes, stream, app);
 }
 
 int gqa_decode_attn_chunked(const void* q, const void* k_cache, const void* v_cache,

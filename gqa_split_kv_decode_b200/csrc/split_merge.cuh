@@ -18,7 +18,7 @@ namespace gqa {
 // Everything a decode kernel needs besides the tensor maps.
 struct DecodeArgs {
   const void* q;            // [B][h_q][D]
-  const void* k;            // packed [rows][h_kv][D] (SIMT path reads it directly)
+  const void* k;            // cache: packed [rows][h_kv][D], or [B][cap][h_kv][D]
   const void* v;
   const int32_t* seqlens;   // [B]
   float* m;                 // triplets: m, l [B*h_q][n_slots], o [B*h_q][n_slots][D]
@@ -26,6 +26,9 @@ struct DecodeArgs {
   float* o;
   float* out;               // fused: [B*h_q][D]
   int* tickets;             // fused: one counter per (b, blockIdx.y)
+  const void* k_new;        // append: the new token's k and v, [B][h_kv][D]; null otherwise
+  const void* v_new;
+  long long cap;            // > 0: cache rows per sequence ([B][cap][h_kv][D]); 0: packed
   int B, h_q, h_kv, G, n_hb;
   int n_splits;             // > 0: split by count
   int chunk_len;            // > 0: split by fixed chunks
@@ -36,31 +39,62 @@ struct DecodeArgs {
 
 enum { kPartial = 0, kFused = 1 };
 
+// Keys of one sequence: `cached` rows are read from the cache; `total` keys
+// are attended, the new token being key number `cached` when appending and
+// the sequence's cache rows have room for it.
+struct SeqKeys {
+  int cached, total;
+  bool append;
+};
+
+__device__ __forceinline__ SeqKeys seq_keys(const DecodeArgs& a, int S) {
+  SeqKeys k;
+  k.cached = S > 0 ? S : 0;
+  if (a.cap > 0 && k.cached > a.cap) k.cached = (int)a.cap;
+  k.append = a.k_new != nullptr && k.cached < a.cap;
+  k.total = k.cached + (k.append ? 1 : 0);
+  return k;
+}
+
+// Reports (once, by the caller's choice of `report`) lengths the call cannot
+// honour: negative, above max_seqlen in chunked mode, above the capacity of a
+// padded cache, or with no room left to append.
+__device__ __forceinline__ void report_length(const DecodeArgs& a, int S, bool report) {
+  if (!report) return;
+  if (S < 0) raise_status(kStatusNegSeqlen);
+  if (a.cap > 0 && (long long)S + (a.k_new ? 1 : 0) > a.cap) raise_status(kStatusSeqlenOverMax);
+}
+
 struct Split {
-  long long off;  // packed row of the sequence's first key
-  int S;          // sequence length (negative lengths read as 0)
+  long long off;  // cache row of the sequence's first key
+  int S;          // keys attended (cached, plus the new token when appending)
   int lo, hi;     // this split's keys [lo, hi), relative to the sequence
+  int cached_hi;  // min(hi, cached keys): the split's keys that come from the cache
+  bool has_new;   // the split holds the appended token (key number `cached`)
   int n_active;   // splits of this sequence that hold keys (>= 1)
 };
 
-// Sequence b's packed offset and the key range of split `slot` (whole warp).
-// Split i covers [i*L, min((i+1)*L, S)) with L = ceil(S / n_splits) or
-// L = chunk_len.  n_active = max(1, ceil(S / L)): the number of splits the
-// fused merge waits for (split 0 stands in for an empty sequence).
+// Sequence b's first cache row and the key range of split `slot` (whole
+// warp).  Split i covers [i*L, min((i+1)*L, S)) with L = ceil(S / n_splits)
+// or L = chunk_len.  n_active = max(1, ceil(S / L)): the number of splits
+// the fused merge waits for (split 0 stands in for an empty sequence).
 __device__ __forceinline__ Split locate_split(const DecodeArgs& a, int b, int slot, int lane,
                                               bool report) {
   long long acc = 0;
-  for (int j = lane; j < b; j += 32) {
-    const int s = __ldg(a.seqlens + j);
-    acc += s > 0 ? s : 0;
-  }
+  if (a.cap > 0) {
+    acc = (long long)b * a.cap;
+  } else {
+    for (int j = lane; j < b; j += 32) {
+      const int s = __ldg(a.seqlens + j);
+      acc += s > 0 ? s : 0;
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-  int S = __ldg(a.seqlens + b);
-  if (S < 0) {
-    if (report) raise_status(kStatusNegSeqlen);
-    S = 0;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
   }
+  const int Sraw = __ldg(a.seqlens + b);
+  report_length(a, Sraw, report);
+  const SeqKeys kk = seq_keys(a, Sraw);
+  const int S = kk.total;
   const long long L =
       a.n_splits > 0 ? ((long long)S + a.n_splits - 1) / a.n_splits : (long long)a.chunk_len;
   int n_active = S > 0 ? (int)(((long long)S + L - 1) / L) : 1;
@@ -77,6 +111,8 @@ __device__ __forceinline__ Split locate_split(const DecodeArgs& a, int b, int sl
   sp.S = S;
   sp.lo = (int)lo;
   sp.hi = (int)hi;
+  sp.cached_hi = (int)(hi < kk.cached ? hi : kk.cached);
+  sp.has_new = kk.append && lo <= kk.cached && kk.cached < hi;
   sp.n_active = n_active;
   return sp;
 }

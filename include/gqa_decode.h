@@ -148,6 +148,30 @@ GQA_API int gqa_decode_attn_noalloc(const void *q, const void *k_cache, const vo
                                     float scale, int dtype, void *stream);
 
 /*
+ * Append-and-attend, the step just before decode attention in a decode loop
+ * (the tt-metal "[Llama2] Perf burndown" page's `update_cache`), fused into
+ * the attention call: the new token's k and v (k_new, v_new: [B][h_kv][d_head],
+ * dtype) are written into the cache at row S_b of each sequence, and the query
+ * attends over the S_b + 1 keys, the new one included.
+ *
+ * The cache is padded, not packed: k_cache, v_cache are [B][cache_capacity]
+ * [h_kv][d_head] and sequence b's key j is row b * cache_capacity + j, so
+ * there is room to append.  Requires S_b + 1 <= cache_capacity; a sequence
+ * without room is attended over its cached rows only and reported as
+ * GQA_ERR_DEVICE_SEQLEN in the status word.  seqlens is NOT advanced: the
+ * caller adds 1 for the next step.  The split of the S_b + 1 keys, the
+ * workspace and the result are as for gqa_decode_attn.  Only the new rows
+ * are written; no other cache row is read or written outside [0, S_b + 1)
+ * of each sequence, except that rows of the previous sequence's unused tail
+ * may be read into a masked, zeroed tile.
+ */
+GQA_API int gqa_decode_attn_append(const void *q, const void *k_new, const void *v_new,
+                                   void *k_cache, void *v_cache, const int32_t *seqlens,
+                                   float *out, int B, int h_q, int h_kv, int d_head,
+                                   int cache_capacity, int n_splits, float scale, int dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Fused decode attention with fixed-length chunks (ragged batches): split i
  * of sequence b covers [i*chunk_len, min((i+1)*chunk_len, S_b)); the last
  * chunk may be partial.  max_seqlen bounds every S_b (host-known, so no
