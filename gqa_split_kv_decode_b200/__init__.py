@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
-    "get_status", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
 
@@ -62,6 +62,7 @@ _partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _
                         _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
 _merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
 _get_status = _sig("gqa_decode_get_status", _ci, _vp)
+_auto_splits = _sig("gqa_decode_auto_splits", _ci, _ci, _ci, _ci, _ci, _ci)
 _launches = _sig("gqa_decode_launches_per_call", _ci, _ci, _ci, _ci, _ci, _ci, _ci)
 _set_timeout = _sig("gqa_decode_set_wait_timeout_ns", _ci, _ull)
 _selftest = _sig("gqa_decode_selftest_wait_timeout", _ci, _ull, _vp)
@@ -288,6 +289,17 @@ def mlo_merge(m, l, o, out=None) -> torch.Tensor:
         _check(_merge(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
                       _stream(m.device)), "mlo_merge")
     return out
+
+
+def auto_splits(B, h_q, h_kv, d, max_seqlen=0, device=None) -> int:
+    """Split count a fused call with n_splits=0 uses on ``device`` (largest
+    count that fills one wave; >= 256 keys per split when max_seqlen > 0)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        n = _auto_splits(B, h_q, h_kv, d, max_seqlen)
+    if n < 0:
+        raise GQADecodeError(-n, "gqa_decode_auto_splits")
+    return n
 
 
 def launches_per_call(B, h_q, h_kv, d, n_slots, dtype=BF16, device=None) -> int:

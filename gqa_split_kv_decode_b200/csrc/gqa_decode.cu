@@ -272,6 +272,30 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
   return launch_simt_hb<64, MODE>(a, hb, grid, st);
 }
 
+// Split count chosen for the caller (n_splits == 0 on a fused call): the
+// largest count whose grid still fits on the GPU in one wave (R CTAs), capped
+// so a split keeps >= 256 keys when max_seqlen is known (> 0).  One wave
+// avoids the grids just past R, where a few leftover splits run alone.
+int auto_splits(int B, int h_q, int h_kv, int D, int max_seqlen) {
+  if (B < 1 || h_kv < 1 || h_q < h_kv || h_q % h_kv) return -GQA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return -GQA_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return -GQA_ERR_CUDA;
+  const int smem = D == 128 ? tc_dynamic_smem<128, kTcWarps, kTcStages>()
+                            : tc_dynamic_smem<64, kTcWarps, kTcStages>();
+  const long long R = (long long)sms * ((228 * 1024) / (smem + 1024));
+  const int G = h_q / h_kv;
+  const long long bh = (long long)B * h_kv * (G <= 16 ? 1 : (G + 15) / 16);
+  long long n = bh >= R ? 1 : R / bh;
+  if (max_seqlen > 0) {
+    const long long cap = (max_seqlen + 255) / 256;
+    if (n > cap) n = cap;
+  }
+  if (n < 1) n = 1;
+  if (n > kMaxSlots) n = kMaxSlots;
+  return (int)n;
+}
+
 // ------------------------------------------------------------ validation
 
 struct Shape {
@@ -515,6 +539,10 @@ const char* gqa_decode_error_string(int status) {
 }
 
 size_t gqa_decode_workspace_size(int B, int h_q, int h_kv, int d_head, int n_splits) {
+  if (n_splits == 0 && B > 0) {
+    n_splits = auto_splits(B, h_q, h_kv, d_head, 0);
+    if (n_splits < 0) return 0;
+  }
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, 1.f, GQA_BF16);
   if (check_shape(s) || n_tickets(s) * sizeof(int) > kTicketBytes) return 0;
   return ws_layout(s).total;
@@ -531,6 +559,10 @@ int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* seqlens, float* out, int B, int h_q, int h_kv, int d_head,
                     int n_splits, float scale, int dtype, void* workspace, size_t workspace_bytes,
                     void* stream) {
+  if (n_splits == 0 && B > 0) {
+    n_splits = auto_splits(B, h_q, h_kv, d_head, 0);
+    if (n_splits < 0) return -n_splits;
+  }
   return fused(q, k_cache, v_cache, seqlens, out,
                split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype), workspace,
                workspace_bytes, stream);
@@ -539,6 +571,10 @@ int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
 int gqa_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* seqlens, float* out, int B, int h_q, int h_kv,
                             int d_head, int n_splits, float scale, int dtype, void* stream) {
+  if (n_splits == 0 && B > 0) {
+    n_splits = auto_splits(B, h_q, h_kv, d_head, 0);
+    if (n_splits < 0) return -n_splits;
+  }
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype);
   if (int rc = check_common(q, k_cache, v_cache, seqlens, s)) return rc;
   if (n_tickets(s) * sizeof(int) > kTicketBytes) return GQA_ERR_UNSUPPORTED;
@@ -560,6 +596,10 @@ int gqa_decode_attn_append(const void* q, const void* k_new, const void* v_new, 
                            void* v_cache, const int32_t* seqlens, float* out, int B, int h_q,
                            int h_kv, int d_head, int cache_capacity, int n_splits, float scale,
                            int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_splits == 0 && B > 0) {
+    n_splits = auto_splits(B, h_q, h_kv, d_head, cache_capacity);
+    if (n_splits < 0) return -n_splits;
+  }
   const Shape s = split_shape(B, h_q, h_kv, d_head, n_splits, scale, dtype);
   if (cache_capacity < 1) return GQA_ERR_INVALID_ARG;
   if ((long long)B * cache_capacity > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;  // int32 rows
@@ -610,6 +650,10 @@ int mlo_merge(const float* m, const float* l, const float* o, float* out, int ro
   if (d_head <= 128)
     return launch_pdl(mlo_merge_kernel<4>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
   return launch_pdl(mlo_merge_kernel<8>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
+}
+
+int gqa_decode_auto_splits(int B, int h_q, int h_kv, int d_head, int max_seqlen) {
+  return auto_splits(B, h_q, h_kv, d_head, max_seqlen);
 }
 
 int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slots, int dtype) {

@@ -47,6 +47,7 @@
  *   nonzero gqa_status and launches nothing.  Supported: d_head in {64, 128};
  *   h_q % h_kv == 0; 1 <= n_splits <= 1024 (n_slots <= 1024 when chunked);
  *   finite scale; dtype GQA_F32 or GQA_BF16 (q, k and v share it).
+ *   n_splits = 0 on a fused call picks the count (gqa_decode_auto_splits).
  * - Errors that only the device can see (a negative S_b, S_b above
  *   max_seqlen in chunked mode, a bounded wait that ran out) set bits of a
  *   per-device status word, read and cleared by gqa_decode_get_status().
@@ -213,6 +214,17 @@ GQA_API int gqa_decode_partial_chunked(const void *q, const void *k_cache, const
  */
 GQA_API int mlo_merge(const float *m, const float *l, const float *o, float *out,
               int rows, int n_splits, int d_head, void *stream);
+
+/*
+ * Split count the library would choose: the largest n_splits whose grid
+ * (n_splits x kv heads x head blocks x B CTAs) still fits on the current
+ * device in one wave, capped so a split keeps at least 256 keys when
+ * max_seqlen > 0 (0: unknown).  Passing n_splits = 0 to gqa_decode_attn,
+ * gqa_decode_attn_noalloc, gqa_decode_attn_append or
+ * gqa_decode_workspace_size makes that choice for the call (the append call
+ * caps with its cache capacity).  Returns n >= 1, or a negative gqa_status.
+ */
+GQA_API int gqa_decode_auto_splits(int B, int h_q, int h_kv, int d_head, int max_seqlen);
 
 /*
  * Number of kernels one fused call (gqa_decode_attn / _chunked / _noalloc)

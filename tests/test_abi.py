@@ -72,7 +72,7 @@ FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation
     (dict(h_q=6, h_kv=4), INVALID),          # h_q not a multiple of h_kv
     (dict(d=96), UNSUPPORTED),               # head dim other than 64 / 128
     (dict(d=0), INVALID),
-    (dict(n_splits=0), INVALID),
+    (dict(n_splits=-1), INVALID),
     (dict(n_splits=1025), INVALID),
     (dict(scale=float("inf")), INVALID),
     (dict(scale=float("nan")), INVALID),

@@ -288,7 +288,7 @@ def test_binding_rejects_bad_tensors(gk):
     with pytest.raises(ValueError):
         gk.gqa_decode_attn(q.transpose(0, 1), k, v, sl, 2)
     with pytest.raises(gk.GQADecodeError) as e:
-        gk.gqa_decode_attn(q, k, v, sl, 0)
+        gk.gqa_decode_attn(q, k, v, sl, -1)
     assert e.value.status == 1
 
 

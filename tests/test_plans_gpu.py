@@ -88,3 +88,24 @@ def test_persistent_reports_bad_lengths(gk):
     sl[1] = 200
     out = gk.gqa_decode_attn_chunked(q, k, v, sl, 16, 256, w.cfg.scale)  # 400 > 256
     assert gk.get_status() == gk.ERR_DEVICE_SEQLEN
+
+
+@pytest.mark.parametrize("case", [(8, 64, 8, 128, 8192), (1, 32, 32, 128, 4096), (3, 16, 2, 64, 700)])
+def test_auto_split_count(gk, case):
+    """n_splits = 0 picks the largest count that fits one wave; the result is
+    the oracle's whatever the count."""
+    B, hq, hkv, d, S = case
+    n = gk.auto_splits(B, hq, hkv, d)
+    assert 1 <= n <= 1024
+    assert gk.launches_per_call(B, hq, hkv, d, n) == 1       # one wave: one launch
+    assert gk.auto_splits(B, hq, hkv, d, max_seqlen=300) <= 2  # >= 256 keys per split
+    w = random_case(B, hq, hkv, d, [S] * B if B > 1 else [S], dtype="bf16", seed=B + S)
+    q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
+    out = gk.gqa_decode_attn(q, k, v, sl, 0, w.cfg.scale)
+    torch.cuda.synchronize()
+    assert gk.get_status() == 0
+    if B * S <= 4096:
+        _check(out, w)
+    else:  # large: compare with the configured count instead of the slow oracle
+        ref = gk.gqa_decode_attn(q, k, v, sl, 8, w.cfg.scale)
+        assert torch.allclose(out, ref, atol=1e-4, rtol=1e-3)
