@@ -109,3 +109,31 @@ def test_auto_split_count(gk, case):
     else:  # large: compare with the configured count instead of the slow oracle
         ref = gk.gqa_decode_attn(q, k, v, sl, 8, w.cfg.scale)
         assert torch.allclose(out, ref, atol=1e-4, rtol=1e-3)
+
+
+@pytest.mark.parametrize("n_splits", [4, 16])   # one wave / persistent plan on a B200
+def test_fused_call_replays_in_a_cuda_graph(gk, n_splits):
+    """A fused call with an explicit workspace and output captures into a CUDA
+    graph (no host synchronisation, no allocation) and replays with new
+    inputs copied into the captured buffers."""
+    B, hq, hkv, d = 4, 64, 8, 128
+    w = random_case(B, hq, hkv, d, [900, 40, 2000, 1], dtype="bf16", seed=31)
+    q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
+    out = torch.empty(B, hq, d, device="cuda")
+    ws = torch.zeros(gk.workspace_size(B, hq, hkv, d, n_splits), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up off the capture
+        gk.gqa_decode_attn(q, k, v, sl, n_splits, w.cfg.scale, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gk.gqa_decode_attn(q, k, v, sl, n_splits, w.cfg.scale, out=out, workspace=ws)
+    for seed in range(3):
+        q.copy_(torch.randn(B, hq, d, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = gk.gqa_decode_attn(q, k, v, sl, n_splits, w.cfg.scale)
+        assert torch.allclose(out, ref, atol=0, rtol=0)
+    assert gk.get_status() == 0
