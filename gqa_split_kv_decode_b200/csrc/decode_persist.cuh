@@ -33,77 +33,74 @@ struct Unit {
 };
 
 // Non-empty splits of a sequence attending S keys: ceil(S / L), clipped to
-// n_slots (0 when S == 0).  L as in locate_split.
-__device__ __forceinline__ int active_splits(const DecodeArgs& a, int S, long long& L) {
+// n_slots (0 when S == 0).  L as in locate_split.  32-bit: S < 2^31 and the
+// host keeps every unit and cache-row count below 2^31.
+__device__ __forceinline__ int active_splits(const DecodeArgs& a, int S, int& L) {
   if (S <= 0) {
     L = 1;
     return 0;
   }
-  L = a.n_splits > 0 ? ((long long)S + a.n_splits - 1) / a.n_splits : (long long)a.chunk_len;
-  long long n = ((long long)S + L - 1) / L;
-  return (int)(n < a.n_slots ? n : a.n_slots);
+  L = a.n_splits > 0 ? (int)(((unsigned)S + a.n_splits - 1) / (unsigned)a.n_splits) : a.chunk_len;
+  const int n = (int)(((unsigned)S + L - 1) / (unsigned)L);
+  return n < a.n_slots ? n : a.n_slots;
 }
 
-__device__ __forceinline__ long long warp_incl_scan(long long v, int lane) {
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long x = __shfl_up_sync(kFull, v, o);
+    const int x = __shfl_up_sync(kFull, v, o);
     if (lane >= o) v += x;
   }
   return v;
 }
 
-// Total number of units (whole warp).
-__device__ long long count_units(const DecodeArgs& a, int H, int lane) {
-  long long total = 0;
-  for (int base = 0; base < a.B; base += 32) {
-    const int b = base + lane;
-    long long L;
-    const int n = b < a.B ? active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L) : 0;
-    total += __shfl_sync(kFull, warp_incl_scan((long long)H * n, lane), 31);
-  }
-  return total;
-}
-
-// Unit u, 0 <= u < count_units (whole warp): scan the sequences for the one
-// holding u, then split u's remainder into (kv head / head block, split).
-__device__ Unit unit_at(const DecodeArgs& a, int H, long long u, int lane) {
-  long long units = 0, rows = 0;
+// One pass over the sequences (whole warp): the number of units, and -- when
+// u < that number -- unit u itself.  A unit is a non-empty split of one
+// (b, kv head / head block); units are numbered b-major, then kv head / head
+// block, then split.
+__device__ Unit scan_units(const DecodeArgs& a, int H, int u, int lane, int* total) {
+  int units = 0, rows = 0;
+  Unit x{};
+  bool found = false;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
     const SeqKeys kk = seq_keys(a, b < a.B ? __ldg(a.seqlens + b) : 0);
-    long long L;
+    int L;
     const int n = b < a.B ? active_splits(a, kk.total, L) : 0;
-    const long long cu = (long long)H * n, cr = kk.cached;
-    const long long iu = warp_incl_scan(cu, lane), ir = warp_incl_scan(cr, lane);
-    const unsigned hit = __ballot_sync(kFull, units + iu > u);
+    const int cu = H * n, cr = kk.cached;
+    const int iu = warp_incl_scan(cu, lane), ir = warp_incl_scan(cr, lane);
+    const unsigned hit = found ? 0u : __ballot_sync(kFull, units + iu > u);
     if (hit) {
       const int j = __ffs(hit) - 1;
-      Unit x;
+      found = true;
       x.b = base + j;
-      const long long r = u - (units + __shfl_sync(kFull, iu - cu, j));
-      x.off = a.cap > 0 ? (long long)x.b * a.cap : rows + __shfl_sync(kFull, ir - cr, j);
+      const int r = u - (units + __shfl_sync(kFull, iu - cu, j));
+      x.off = a.cap > 0 ? (long long)x.b * a.cap : (long long)rows + __shfl_sync(kFull, ir - cr, j);
       const int St = __shfl_sync(kFull, kk.total, j), Sc = __shfl_sync(kFull, kk.cached, j);
-      const bool app = __shfl_sync(kFull, kk.append, j);
-      long long Lj;
-      const int nj = active_splits(a, St, Lj);
-      x.gy = (int)(r / nj);
-      x.slot = (int)(r - (long long)x.gy * nj);
-      long long lo = (long long)x.slot * Lj, hi = lo + Lj;
-      if (hi > St) hi = St;
-      x.lo = (int)lo;
-      x.hi = (int)hi;
-      x.cached_hi = (int)(hi < Sc ? hi : Sc);
+      const bool app = __shfl_sync(kFull, (int)kk.append, j) != 0;
+      const int nj = __shfl_sync(kFull, n, j), Lj = __shfl_sync(kFull, L, j);
+      x.gy = r / nj;
+      x.slot = r - x.gy * nj;
+      const int lo = x.slot * Lj;
+      const int hi = (St - lo < Lj) ? St : lo + Lj;
+      x.lo = lo;
+      x.hi = hi;
+      x.cached_hi = hi < Sc ? hi : Sc;
       x.has_new = app && lo <= Sc && Sc < hi;
-      const long long len = x.cached_hi > x.lo ? x.cached_hi - x.lo : 0;
-      x.ntiles = (int)((len + kTileKeys - 1) / kTileKeys);
-      return x;
+      const int len = x.cached_hi > x.lo ? x.cached_hi - x.lo : 0;
+      x.ntiles = (len + kTileKeys - 1) / kTileKeys;
+      if (!total) return x;
     }
     units += __shfl_sync(kFull, iu, 31);
     rows += __shfl_sync(kFull, ir, 31);
   }
-  Unit none{};  // not reached for u < count_units
-  return none;
+  if (total) *total = units;
+  return x;
+}
+
+// Unit u, 0 <= u < the number of units (whole warp).
+__device__ __forceinline__ Unit unit_at(const DecodeArgs& a, int H, long long u, int lane) {
+  return scan_units(a, H, (int)u, lane, nullptr);
 }
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
@@ -211,10 +208,22 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
 
-  const long long A = count_units(a, H, lane);
+  int A32 = 0;
+  const Unit first = scan_units(a, H, blockIdx.x, lane, &A32);  // count + first unit, one pass
+  const long long A = A32;
   const uint64_t policy = l2_policy_evict_first();
   const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
   const uint32_t bar0 = smem_u32(&full_bar[warp * NS]);
+
+  // q of the first unit is requested before any K/V tile, so it is not
+  // queued behind the whole grid's first burst of TMA traffic.
+  uint32_t qf[NT][STEPS][2];
+  int q_b = -1, q_gy = -1;
+  if (blockIdx.x < A) {
+    load_q_frags<D, NT>(qf, a, first.b, first.gy / a.n_hb, first.gy % a.n_hb, lane);
+    q_b = first.b;
+    q_gy = first.gy;
+  }
 
   // ---- issue cursor: the next tile of this warp's sequence (warp-uniform)
   long long ia = blockIdx.x;
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(NW * 32)
   int it = warp;
   bool more = false;
   if (ia < A) {
-    iu = unit_at(a, H, ia, lane);
+    iu = first;
     more = true;
     while (more && it >= iu.ntiles) {  // no tile of this unit for this warp
       ia += gridDim.x;
@@ -257,13 +266,11 @@ __global__ void __launch_bounds__(NW * 32)
   for (int s = 0; s < NS && more; ++s) issue_next();
   __syncwarp();
 
-  uint32_t qf[NT][STEPS][2];
-  int q_b = -1, q_gy = -1;
   WarpAcc<D, NT> acc;
   bool failed = false;
 
   for (long long u = blockIdx.x; u < A; u += gridDim.x) {
-    const Unit cu = unit_at(a, H, u, lane);
+    const Unit cu = u == blockIdx.x ? first : unit_at(a, H, u, lane);
     const int g = cu.gy / a.n_hb, hb = cu.gy % a.n_hb;
     if (cu.b != q_b || cu.gy != q_gy) {
       load_q_frags<D, NT>(qf, a, cu.b, g, hb, lane);
@@ -361,7 +368,7 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const DecodeArgs a, int
   const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= (long long)a.B * a.h_q) return;
   const int b = (int)(row / a.h_q);
-  long long L;
+  int L;
   const int n = active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L);
   const int lane = threadIdx.x & 31;
   float* out = a.out + row * D;

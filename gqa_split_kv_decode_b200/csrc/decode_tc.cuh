@@ -363,6 +363,10 @@ __global__ void __launch_bounds__(NW * 32)
                       static_cast<int>(sp.off + tile_row0(t)), policy);
   };
 
+  // q is requested before any K/V tile, so it is not queued behind the
+  // grid's first burst of TMA traffic.
+  uint32_t qf[NT][STEPS][2];
+  load_q_frags<D, NT>(qf, a, b, g, hb, lane);
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
@@ -371,9 +375,6 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
   __syncwarp();
-
-  uint32_t qf[NT][STEPS][2];
-  load_q_frags<D, NT>(qf, a, b, g, hb, lane);
   WarpAcc<D, NT> acc;
   acc.reset();
 
