@@ -52,6 +52,8 @@ class Oracle:
         lib.oracle_partials.restype = ci
         lib.oracle_merge.argtypes = [f64p, f64p, f64p, ci, ci, ci, f64p]
         lib.oracle_merge.restype = None
+        lib.oracle_prefill.argtypes = [vp, vp, vp, i32p, ci, ci, ci, ci, cd, ci, i32p, ci, ci, f64p]
+        lib.oracle_prefill.restype = ci
         self.lib = lib
         self.path = path
 
@@ -63,6 +65,9 @@ class Oracle:
 
     def merge(self, *a, **kw):
         return _merge(self.lib, *a, **kw)
+
+    def prefill(self, *a, **kw):
+        return _prefill(self.lib, *a, **kw)
 
 
 def compile_variant(src_text: str, out_path: str) -> Oracle:
@@ -133,6 +138,35 @@ def partials(*a, **kw):
 
 def merge(*a, **kw):
     return default().merge(*a, **kw)
+
+
+def prefill(*a, **kw):
+    return default().prefill(*a, **kw)
+
+
+def _prefill(lib, q, k, v, seqlens, h_q: int, h_kv: int, scale: float, items=None, nthreads: int = 0):
+    """Causal prefill output in fp64.
+
+    q: packed [sum S_b, h_q, d]; k, v: packed [sum S_b, h_kv, d]; seqlens
+    int32 [B].  ``items`` selects (b, h, i) triples -- query position i of
+    sequence b, head h (default: all, in (b, i, h) order, i.e. q's row
+    order).  Returns float64 [n_items, d]."""
+    qa, dt = _raw(q)
+    ka, _ = _raw(k)
+    va, _ = _raw(v)
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    B = sl.shape[0]
+    d = qa.shape[-1]
+    if items is None:
+        items = [(b, h, i) for b in range(B) for i in range(int(sl[b])) for h in range(h_q)]
+    it = np.ascontiguousarray(np.asarray(items, dtype=np.int32).reshape(-1, 3))
+    out = np.zeros((it.shape[0], d), dtype=np.float64)
+    rc = lib.oracle_prefill(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, _ptr(sl, ctypes.c_int32),
+                            B, h_q, h_kv, d, float(scale), dt, _ptr(it, ctypes.c_int32), it.shape[0],
+                            nthreads, _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise ValueError("oracle_prefill: bad arguments")
+    return out
 
 
 def _attn(lib, q, k, v, seqlens, h_q: int, h_kv: int, scale: float, items=None, nthreads: int = 0):

@@ -41,6 +41,10 @@
  *   - Split i of a sequence of length S covers [i*L, min((i+1)*L, S)) with
  *     L = ceil(S / n_splits), or L = chunk_len in chunked mode.
  *
+ * Prefill (causal, every position of a sequence is a query): query i of
+ * sequence b (q row S_0 + ... + S_{b-1} + i) attends keys j <= i of the same
+ * sequence -- the definition above with S_b replaced by i + 1.
+ *
  * Everything is two-pass and unsplit: logits are stored, the maximum is taken,
  * then exponentials and sums are formed in fp64 from the exact fp64 values of
  * the stored fp32 / bf16 inputs.
@@ -72,16 +76,19 @@ typedef struct {
     const int32_t *seqlens;
     const int64_t *row_off; /* packed row offset of each sequence */
     int B, h_q, h_kv, d, dtype;
+    int causal;             /* prefill: q holds every position; items are (b, h, i) */
     double scale;
     /* split policy: n_splits > 0 -> L = ceil(S/n_splits); else chunk_len */
     int n_splits, chunk_len, n_out_splits;
 } problem;
 
-/* Logit s_j for query (b, h) and key j of sequence b. */
-static double logit(const problem *p, int b, int h, int64_t j) {
+/* Logit s_j for query (b, h) -- at position i of the sequence when causal --
+ * and key j of sequence b. */
+static double logit_at(const problem *p, int b, int h, int64_t i, int64_t j) {
     int G = p->h_q / p->h_kv;
     int g = h / G;
-    int64_t qi = ((int64_t)b * p->h_q + h) * p->d;
+    int64_t qrow = p->causal ? p->row_off[b] + i : (int64_t)b;
+    int64_t qi = (qrow * p->h_q + h) * p->d;
     int64_t ki = ((p->row_off[b] + j) * p->h_kv + g) * p->d;
     double acc = 0.0;
     for (int t = 0; t < p->d; ++t)
@@ -89,10 +96,12 @@ static double logit(const problem *p, int b, int h, int64_t j) {
     return p->scale * acc;
 }
 
+static double logit(const problem *p, int b, int h, int64_t j) { return logit_at(p, b, h, 0, j); }
+
 /* Triplet of (b, h) over keys [lo, hi): the plain two-pass definition.
  * Writes m, l and o[0..d). */
-static void range_triplet(const problem *p, int b, int h, int64_t lo, int64_t hi,
-                          double *s_buf, double *m_out, double *l_out, double *o_out) {
+static void range_triplet_at(const problem *p, int b, int h, int64_t i, int64_t lo, int64_t hi,
+                             double *s_buf, double *m_out, double *l_out, double *o_out) {
     int G = p->h_q / p->h_kv;
     int g = h / G;
     for (int t = 0; t < p->d; ++t) o_out[t] = 0.0;
@@ -104,7 +113,7 @@ static void range_triplet(const problem *p, int b, int h, int64_t lo, int64_t hi
     /* pass 1: logits and their maximum */
     double M = -INFINITY;
     for (int64_t j = lo; j < hi; ++j) {
-        double s = logit(p, b, h, j);
+        double s = logit_at(p, b, h, i, j);
         s_buf[j - lo] = s;
         if (s > M) M = s;
     }
@@ -120,6 +129,11 @@ static void range_triplet(const problem *p, int b, int h, int64_t lo, int64_t hi
     *l_out = l;
 }
 
+static void range_triplet(const problem *p, int b, int h, int64_t lo, int64_t hi,
+                          double *s_buf, double *m_out, double *l_out, double *o_out) {
+    range_triplet_at(p, b, h, 0, lo, hi, s_buf, m_out, l_out, o_out);
+}
+
 /* ---- work distribution over (b, h) items ------------------------------ */
 
 typedef struct {
@@ -128,7 +142,7 @@ typedef struct {
     int n_items;
     int next;             /* shared cursor */
     pthread_mutex_t lock;
-    int mode;             /* 0 = full attention, 1 = partials */
+    int mode;             /* 0 = full attention, 1 = partials, 2 = causal prefill */
     double *out;          /* mode 0: [n_items][d] */
     double *m, *l, *o;    /* mode 1: [n_items][n_out_splits](x d) */
     int64_t max_len;
@@ -158,6 +172,14 @@ static void *worker(void *arg) {
     double *o_tmp = (double *)malloc(sizeof(double) * (size_t)p->d);
     int it;
     while ((it = take(jb)) >= 0) {
+        if (jb->mode == 2) {
+            int b = jb->items[3 * it], h = jb->items[3 * it + 1], i = jb->items[3 * it + 2];
+            double m, l;
+            range_triplet_at(p, b, h, i, 0, (int64_t)i + 1, s_buf, &m, &l, o_tmp);
+            double *dst = jb->out + (int64_t)it * p->d;
+            for (int t = 0; t < p->d; ++t) dst[t] = o_tmp[t] / l;
+            continue;
+        }
         int b = jb->items[2 * it], h = jb->items[2 * it + 1];
         int64_t S = p->seqlens[b];
         if (jb->mode == 0) {
@@ -193,8 +215,13 @@ static int run(problem *p, const int32_t *items, int n_items, int nthreads, int 
     row_off[p->B] = acc;
     p->row_off = row_off;
     for (int i = 0; i < n_items; ++i) {
-        int b = items[2 * i], h = items[2 * i + 1];
+        int w = mode == 2 ? 3 : 2;
+        int b = items[w * i], h = items[w * i + 1];
         if (b < 0 || b >= p->B || h < 0 || h >= p->h_q) { free(row_off); return 1; }
+        if (mode == 2 && (items[3 * i + 2] < 0 || items[3 * i + 2] >= p->seqlens[b])) {
+            free(row_off);
+            return 1;
+        }
     }
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
     if (nthreads < 1) nthreads = 1;
@@ -275,4 +302,19 @@ void oracle_merge(const double *m, const double *l, const double *o,
         for (int t = 0; t < d; ++t) out[(int64_t)r * d + t] = L > 0.0 ? acc[t] / L : 0.0;
     }
     free(acc);
+}
+
+/* Causal prefill output O[it][d] (fp64) for each listed (b, h, i): query i of
+ * sequence b, head h, over keys 0..i of that sequence.  q, k, v: packed
+ * [sum S_b][heads][d] (q with h_q heads, k and v with h_kv).  Returns 0, or 1
+ * on bad arguments. */
+int oracle_prefill(const void *q, const void *k, const void *v, const int32_t *seqlens,
+                   int B, int h_q, int h_kv, int d, double scale, int dtype,
+                   const int32_t *items, int n_items, int nthreads, double *out) {
+    problem p;
+    memset(&p, 0, sizeof p);
+    p.q = q; p.k = k; p.v = v; p.seqlens = seqlens;
+    p.B = B; p.h_q = h_q; p.h_kv = h_kv; p.d = d; p.dtype = dtype; p.scale = scale;
+    p.causal = 1;
+    return run(&p, items, n_items, nthreads, 2, out, NULL, NULL, NULL);
 }

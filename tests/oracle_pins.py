@@ -331,7 +331,86 @@ def pin_head_permutation(orc):
     assert np.array_equal(got, full[perm])
 
 
+def _sdpa_causal_ref(q, k, v, seqlens, h_q, h_kv, scale):
+    """torch's fp64 causal scaled_dot_product_attention, sequence by sequence,
+    each kv head repeated for its consecutive query heads; rows in q's order."""
+    G = h_q // h_kv
+    off = _offsets(list(seqlens))
+    outs = []
+    for b in range(len(seqlens)):
+        qb = q[off[b]:off[b + 1]].double().permute(1, 0, 2)                      # [h_q, S, d]
+        kb = k[off[b]:off[b + 1]].double().permute(1, 0, 2).repeat_interleave(G, dim=0)
+        vb = v[off[b]:off[b + 1]].double().permute(1, 0, 2).repeat_interleave(G, dim=0)
+        ob = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, is_causal=True, scale=scale)
+        outs.append(ob.permute(1, 0, 2).reshape(-1, q.shape[-1]))                 # [(S, h_q), d]
+    return torch.cat(outs).numpy()
+
+
+def _prefill_case(seqlens, h_q, h_kv, d, dtype, seed, std=1.0):
+    """Packed q [sum S, h_q, d] plus k, v [sum S, h_kv, d]."""
+    w = random_case(len(seqlens), h_q, h_kv, d, seqlens, dtype=dtype, seed=seed, std=std)
+    rows = int(sum(seqlens))
+    g = torch.Generator().manual_seed(seed + 7)
+    q = (torch.randn(rows, h_q, d, generator=g) * std).to(w.k.dtype)
+    return q, w.k, w.v, w.seqlens, w.cfg.scale
+
+
+def pin_prefill_matches_library_causal_sdpa(orc):
+    """Causal prefill against torch's fp64 causal SDPA (MHA and GQA)."""
+    for seqlens, hq, hkv, d in [([33, 7], 4, 4, 64), ([40, 1, 17], 8, 2, 128)]:
+        q, k, v, sl, scale = _prefill_case(seqlens, hq, hkv, d, "bf16", seed=sum(seqlens))
+        got = orc.prefill(q, k, v, sl, hq, hkv, scale)
+        ref = _sdpa_causal_ref(q, k, v, seqlens, hq, hkv, scale)
+        assert np.allclose(got, ref, rtol=1e-11, atol=1e-13), np.abs(got - ref).max()
+
+
+def pin_prefill_decimal_bruteforce(orc):
+    """Tiny causal cases against a 50-digit Decimal brute force."""
+    getcontext().prec = 50
+    seqlens, hq, hkv, d = [3, 2], 4, 2, 4
+    q, k, v, sl, scale = _prefill_case(seqlens, hq, hkv, d, "f32", seed=44)
+    qx, kx, vx = _exact(q), _exact(k), _exact(v)
+    off = _offsets(seqlens)
+    items, ref = [], []
+    for b, S in enumerate(seqlens):
+        for i in range(S):
+            for h in range(hq):
+                g = h // (hq // hkv)
+                s = []
+                for j in range(i + 1):
+                    acc = Decimal(0)
+                    for t in range(d):
+                        acc += Decimal(float(qx[off[b] + i, h, t])) * Decimal(float(kx[off[b] + j, g, t]))
+                    s.append((acc * Decimal(scale)).exp())
+                den = sum(s, Decimal(0))
+                ref.append([float(sum((s[j] * Decimal(float(vx[off[b] + j, g, t])) for j in range(i + 1)),
+                                      Decimal(0)) / den) for t in range(d)])
+                items.append((b, h, i))
+    got = orc.prefill(q, k, v, sl, hq, hkv, scale, items=items)
+    assert np.allclose(got, np.array(ref), rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_first_row_and_last_row(orc):
+    """Position 0 attends only itself: O = v_0.  The last position of a
+    sequence attends every key: it equals decode attention with that query."""
+    seqlens, hq, hkv, d = [25, 9], 8, 2, 64
+    q, k, v, sl, scale = _prefill_case(seqlens, hq, hkv, d, "bf16", seed=45)
+    off = _offsets(seqlens)
+    vx = _exact(v)
+    got0 = orc.prefill(q, k, v, sl, hq, hkv, scale, items=[(b, h, 0) for b in range(2) for h in range(hq)])
+    for b in range(2):
+        for h in range(hq):
+            assert np.array_equal(got0[b * hq + h], vx[off[b], h // 4])
+    last = orc.prefill(q, k, v, sl, hq, hkv, scale,
+                       items=[(b, h, seqlens[b] - 1) for b in range(2) for h in range(hq)])
+    qd = torch.stack([q[off[b + 1] - 1] for b in range(2)])                     # [B, h_q, d]
+    dec = orc.attn(qd, k, v, sl, hq, hkv, scale)
+    assert np.allclose(last, dec, rtol=1e-13, atol=1e-15)
+
+
 PINS = [pin_worked_example, pin_decimal_bruteforce, pin_scale_zero_is_mean,
         pin_constant_keys_is_mean, pin_single_key, pin_dominant_logit,
         pin_gqa_contiguous_mapping, pin_matches_library_sdpa, pin_partial_is_range_softmax,
-        pin_split_merge_invariance, pin_empty_sequences, pin_head_permutation]
+        pin_split_merge_invariance, pin_empty_sequences, pin_head_permutation,
+        pin_prefill_matches_library_causal_sdpa, pin_prefill_decimal_bruteforce,
+        pin_prefill_first_row_and_last_row]

@@ -22,6 +22,10 @@ MUTANTS = [
      "int64_t ki = ((p->row_off[b] + j) * p->h_kv + (h % p->h_kv)) * p->d;"),
     ("ceil_as_floor", "(S + p->n_splits - 1) / p->n_splits", "S / p->n_splits"),
     ("wrong_row_offset", "row_off[b] = acc;", "row_off[b] = b * (int64_t)p->seqlens[0];"),
+    ("prefill_excludes_diagonal", "range_triplet_at(p, b, h, i, 0, (int64_t)i + 1,",
+     "range_triplet_at(p, b, h, i, 0, (int64_t)i + (i == 0),"),
+    ("prefill_query_row_of_first_position", "int64_t qrow = p->causal ? p->row_off[b] + i : (int64_t)b;",
+     "int64_t qrow = p->causal ? p->row_off[b] : (int64_t)b;"),
 ]
 
 
