@@ -5,7 +5,10 @@ PyTorch is used for device memory and the current stream only: every step of
 the computation runs in the library's CUDA kernels.  If the library is
 missing, importing this package raises ImportError -- there is no fallback.
 
-Layouts (see the header): q [B, h_q, d]; k_cache, v_cache packed
+Causal prefill (``include/gqa_prefill.h``): ``gqa_prefill_attn`` with q packed
+[sum S_b, h_q, d], k, v [sum S_b, h_kv, d], out fp32 [sum S_b, h_q, d].
+
+Decode layouts (see the header): q [B, h_q, d]; k_cache, v_cache packed
 [sum S_b, h_kv, d]; seqlens int32 [B] on the device; out fp32 [B, h_q, d];
 triplets m, l [B, h_q, n_slots] and o [B, h_q, n_slots, d] in fp32.
 """
@@ -20,7 +23,7 @@ import torch
 __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
-    "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "gqa_prefill_attn", "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
 
@@ -61,6 +64,8 @@ _partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c
 _partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci,
                         _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
 _merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
+_prefill = _sig("gqa_prefill_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf,
+                _ci, _vp)
 _get_status = _sig("gqa_decode_get_status", _ci, _vp)
 _auto_splits = _sig("gqa_decode_auto_splits", _ci, _ci, _ci, _ci, _ci, _ci)
 _launches = _sig("gqa_decode_launches_per_call", _ci, _ci, _ci, _ci, _ci, _ci, _ci)
@@ -331,3 +336,38 @@ def selftest_wait_timeout(ns: int, device=None) -> None:
 
 def release() -> None:
     _check(_release(), "gqa_decode_release")
+
+
+def gqa_prefill_attn(q, k, v, seqlens, scale=None, max_seqlen=None, out=None):
+    """Causal prefill attention: query i of sequence b attends keys 0..i of
+    that sequence.  q [rows, h_q, 128], k, v [rows, h_kv, 128] bf16, packed by
+    sequence (rows = sum S_b); seqlens int32 [B] on the device.  Returns fp32
+    [rows, h_q, 128].  ``max_seqlen`` bounds every S_b; when omitted it is read
+    from ``seqlens`` (one device-to-host copy)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("seqlens", seqlens)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.device == k.device == v.device == seqlens.device):
+        raise ValueError("all tensors must be on one device")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or q.shape[0] != k.shape[0]:
+        raise ValueError("q must be [rows, h_q, d]; k, v [rows, h_kv, d] with the same rows")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise ValueError("q, k and v must share one dtype")
+    if seqlens.dtype != torch.int32 or seqlens.dim() != 1:
+        raise ValueError("seqlens must be int32 [B]")
+    if q.shape[2] != k.shape[2]:
+        raise ValueError("head dims differ")
+    rows, h_q, d = q.shape
+    B = seqlens.shape[0]
+    if max_seqlen is None:
+        max_seqlen = int(seqlens.max().item()) if B > 0 else 0
+    if out is None:
+        out = torch.empty((rows, h_q, d), dtype=torch.float32, device=q.device)
+    elif out.shape != (rows, h_q, d) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be contiguous fp32 [rows, h_q, d]")
+    _check(_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(seqlens), _ptr(out), B, rows, int(max_seqlen),
+                    h_q, k.shape[1], d, _default_scale(d, scale), _dtype_code(q),
+                    _stream(q.device)), "gqa_prefill_attn")
+    return out

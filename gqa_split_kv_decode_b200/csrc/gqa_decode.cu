@@ -15,9 +15,11 @@
 #include <utility>
 
 #include "gqa_decode.h"
+#include "gqa_prefill.h"
 #include "decode_persist.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "prefill_tc.cuh"
 #include "split_merge.cuh"
 
 namespace {
@@ -517,6 +519,65 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
     raise_status(kStatusTimeout);
 }
 
+// ------------------------------------------------------------ prefill
+
+// 3-D view (d = 128, head, row) of a packed bf16 [rows][heads][128] tensor;
+// box = 64 d x 1 head x 128 rows, 128-byte swizzle.  The row extent is the
+// tensor's own, so a tile that runs past the last row reads zeros.
+bool encode_rows_map(CUtensorMap* map, const void* base, int heads, int rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kPfD), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kPfD) * 2,
+                                 static_cast<cuuint64_t>(heads) * kPfD * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kPfRows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int prefill(const void* q, const void* k, const void* v, const int32_t* seqlens, float* out,
+            int B, int total_rows, int max_seqlen, int h_q, int h_kv, int d_head, float scale,
+            int dtype, void* stream) {
+  if (B < 0 || total_rows < 0 || max_seqlen < 0 || h_q < 1 || h_kv < 1 || h_q % h_kv != 0)
+    return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return GQA_ERR_INVALID_ARG;
+  if (d_head < 1) return GQA_ERR_INVALID_ARG;
+  if (d_head != kPfD || dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if (B == 0 || total_rows == 0) return GQA_OK;
+  if (max_seqlen == 0) return GQA_ERR_INVALID_ARG;   // rows exist, so some S_b > 0
+  if (!q || !k || !v || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(seqlens, 4))
+    return GQA_ERR_INVALID_ARG;
+  const int n_qtiles = (max_seqlen + kPfRows - 1) / kPfRows;
+  if (B > 65535 || h_q > 65535 || n_qtiles > 65535) return GQA_ERR_UNSUPPORTED;
+  static std::atomic<uint64_t> attr_done{0};
+  if (int rc = ensure_smem_attr(prefill_tc_bf16, kPfDynSmem, attr_done)) return rc;
+  CUtensorMap qmap, kmap, vmap;
+  if (!encode_rows_map(&qmap, q, h_q, total_rows) || !encode_rows_map(&kmap, k, h_kv, total_rows) ||
+      !encode_rows_map(&vmap, v, h_kv, total_rows))
+    return GQA_ERR_CUDA;
+  PrefillArgs a{};
+  a.seqlens = seqlens;
+  a.out = out;
+  a.total_rows = total_rows;
+  a.B = B;
+  a.h_q = h_q;
+  a.h_kv = h_kv;
+  a.G = h_q / h_kv;
+  a.n_qtiles = n_qtiles;
+  a.scale_log2 = scale * kLog2e;
+  a.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  return launch_pdl(prefill_tc_bf16, dim3(h_q, B, n_qtiles), dim3(kPfThreads), kPfDynSmem,
+                    as_stream(stream), qmap, kmap, vmap, a);
+}
+
 }  // namespace
 
 // ====================================================================== ABI
@@ -667,6 +728,13 @@ int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slo
   const int plan = fused_plan(units, d_head);
   if (plan < 0) return -GQA_ERR_CUDA;
   return plan == kPlanPersistent ? 2 : 1;
+}
+
+int gqa_prefill_attn(const void* q, const void* k, const void* v, const int32_t* seqlens,
+                     float* out, int B, int total_rows, int max_seqlen, int h_q, int h_kv,
+                     int d_head, float scale, int dtype, void* stream) {
+  return prefill(q, k, v, seqlens, out, B, total_rows, max_seqlen, h_q, h_kv, d_head, scale,
+                 dtype, stream);
 }
 
 int gqa_decode_get_status(void* stream) {

@@ -1,0 +1,431 @@
+// Causal prefill attention (S_q = T > 1) on the fifth-generation tensor
+// cores: the compute-bound counterpart of decode, the "flash-attention style"
+// SDPA of the tt-metal "[Llama2] Perf burndown" page (Prefill 2k list), whose
+// arithmetic intensity grows with T (scaling-book "All About Transformer
+// Inference", the prefill discussion).
+//
+// Query i of sequence b attends keys 0..i of the same sequence:
+//   O_i = sum_{j<=i} e^{s_ij - m_i} v_j / sum_{j<=i} e^{s_ij - m_i},
+//   s_ij = scale <q_i, k_j>,  query head h reading kv head h / (h_q / h_kv).
+//
+// One CTA = 128 query rows of one head of one sequence.  Six warps:
+//   warps 0-3  softmax: thread r owns row r (TMEM lane r) -- reads S from
+//              TMEM, keeps the row's running max and denominator, writes P
+//              (bf16) to shared memory, rescales O in TMEM when needed, and
+//              finally normalises O and stores it;
+//   warp 4     TMA producer: Q once, then K and V tiles of 128 keys through
+//              two-stage rings;
+//   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM S
+//              buffers, then O += P V into the TMEM O accumulator.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384) of a 512-column
+// allocation (fp32, lane = query row).
+//
+// Rows whose whole key range is short (the first 128 positions of a
+// sequence, q-tile 0) take P as two bf16 parts, hi + lo, summed by two MMAs
+// into O, so a row of a few keys keeps near-fp32 weights; longer rows use
+// one bf16 P (its rounding averages out over the keys).
+#pragma once
+
+#include "device_common.cuh"
+#include "tcgen05.cuh"
+
+namespace gqa {
+
+constexpr int kPfRows = 128;      // query rows per CTA (MMA M)
+constexpr int kPfKeys = 128;      // keys per K/V tile (MMA N of QK^T, K of PV)
+constexpr int kPfD = 128;         // head dim (MMA K of QK^T, N of PV)
+constexpr int kPfThreads = 192;
+constexpr int kPfHalfBytes = kPfRows * 128;        // one 64-column half of a 128-row tile
+constexpr int kPfTileBytes = 2 * kPfHalfBytes;     // 32 KiB
+// Shared memory: Q, K[2], V[2], P[2] tiles, 1024-byte aligned.
+constexpr int kPfSmemQ = 0;
+constexpr int kPfSmemK = kPfSmemQ + kPfTileBytes;
+constexpr int kPfSmemV = kPfSmemK + 2 * kPfTileBytes;
+constexpr int kPfSmemP = kPfSmemV + 2 * kPfTileBytes;
+constexpr int kPfSmemBytes = kPfSmemP + 2 * kPfTileBytes;   // 224 KiB
+constexpr int kPfDynSmem = kPfSmemBytes + 1024;            // + alignment slack
+constexpr uint32_t kPfTmemCols = 512;
+constexpr uint32_t kPfColS0 = 0, kPfColS1 = 128, kPfColO = 256;
+constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale: keep the max unless it grew by > 2^8
+
+struct PrefillArgs {
+  const int32_t* seqlens;   // [B] device
+  float* out;               // [total_rows][h_q][128] fp32
+  long long total_rows;     // rows of the packed q / k / v (sum of S_b)
+  int B, h_q, h_kv, G;      // G = h_q / h_kv
+  int n_qtiles;             // ceil(max_seqlen / 128): the grid's tile extent
+  float scale_log2;         // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+// Barriers of one CTA (shared memory).
+struct PfBars {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], pv_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint64_t& b) { return smem_u32(&b); }
+
+// Bounded wait shared by every role: false (and the CTA's abort flag set,
+// the timeout recorded) when the wait ran out or another role gave up.
+__device__ __forceinline__ bool pf_wait(PfBars& sb, uint64_t& bar, uint32_t parity,
+                                        unsigned long long timeout_ns) {
+  if (*reinterpret_cast<volatile int*>(&sb.abort)) return false;
+  if (mbar_wait_bounded(bar_addr(bar), parity, timeout_ns)) return true;
+  *reinterpret_cast<volatile int*>(&sb.abort) = 1;
+  raise_status(kStatusTimeout);
+  return false;
+}
+
+// Warp-uniform version for the softmax warps (their TMEM accesses are
+// warp-collective, so every lane must take the same branch).
+__device__ __forceinline__ bool pf_wait_warp(PfBars& sb, uint64_t& bar, uint32_t parity,
+                                             unsigned long long timeout_ns) {
+  const bool ok = pf_wait(sb, bar, parity, timeout_ns);
+  return __all_sync(kFull, ok);
+}
+
+// Loads a 128-row x 128-column bf16 tile as two 64-column boxes (128-byte
+// swizzle): columns [0,64) at dst, [64,128) at dst + 16 KiB.
+__device__ __forceinline__ void pf_load_tile(uint32_t dst, const CUtensorMap* map, int head,
+                                             long long row, uint32_t bar, uint64_t policy) {
+  mbar_arrive_expect_tx(bar, kPfTileBytes);
+  tma_load_3d(dst, map, 0, head, (int)row, bar, policy);
+  tma_load_3d(dst + kPfHalfBytes, map, 64, head, (int)row, bar, policy);
+}
+
+// Warp 4, one thread: Q, then K_j / V_j for j = 0 .. nt-1 through the rings.
+// Stage s = j & 1 is refilled once the MMA that read its previous tile
+// (S_{j-2} for K, PV_{j-2} for V) has completed.  At the end it waits for
+// every copy it issued, so none lands after the CTA has gone.
+__device__ __forceinline__ void pf_producer(PfBars& sb, uint32_t smem, const CUtensorMap* qmap,
+                                            const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                            int h, int g, long long qrow, long long krow0, int nt,
+                                            unsigned long long tmo) {
+  const uint64_t pol_q = l2_policy_evict_first();
+  const uint64_t pol_kv = l2_policy_evict_last();
+  pf_load_tile(smem + kPfSmemQ, qmap, h, qrow, bar_addr(sb.q_full), pol_q);
+  int issued = 0;
+  for (int j = 0; j < nt; ++j) {
+    const int s = j & 1;
+    const uint32_t par = ((j >> 1) - 1) & 1;
+    const long long row = krow0 + (long long)j * kPfKeys;
+    if (j >= 2 && !pf_wait(sb, sb.k_empty[s], par, tmo)) break;
+    pf_load_tile(smem + kPfSmemK + s * kPfTileBytes, kmap, g, row, bar_addr(sb.k_full[s]), pol_kv);
+    if (j >= 2 && !pf_wait(sb, sb.v_empty[s], par, tmo)) {
+      issued = 2 * j + 1;
+      break;
+    }
+    pf_load_tile(smem + kPfSmemV + s * kPfTileBytes, vmap, g, row, bar_addr(sb.v_full[s]), pol_kv);
+    issued = 2 * j + 2;
+  }
+  // Drain: the last K and V load of each stage (earlier ones are implied,
+  // since a stage is refilled only after its previous load was consumed).
+  mbar_wait_bounded(bar_addr(sb.q_full), 0, tmo);
+  for (int n = issued - 1; n >= 0 && n >= issued - 4; --n) {
+    const int j = n >> 1;
+    uint64_t& bar = (n & 1) ? sb.v_full[j & 1] : sb.k_full[j & 1];
+    if (!mbar_wait_bounded(bar_addr(bar), (j >> 1) & 1, tmo)) raise_status(kStatusTimeout);
+  }
+}
+
+// S_j = Q K_j^T (M = 128 rows, N = 128 keys, K = 128 head dims): eight
+// K = 16 steps; both operands K-major, each step 32 bytes further along the
+// swizzled 128-byte rows, the second 64 dims in the tile's second half.
+__device__ __forceinline__ void pf_issue_qk(uint32_t smem, uint32_t tmem, int j) {
+  constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfKeys, false);
+  const uint32_t qa = smem + kPfSmemQ;
+  const uint32_t kb = smem + kPfSmemK + (j & 1) * kPfTileBytes;
+  const uint32_t d = tmem + ((j & 1) ? kPfColS1 : kPfColS0);
+#pragma unroll
+  for (int k = 0; k < kPfD / 16; ++k) {
+    const uint32_t off = (k >> 2) * kPfHalfBytes + (k & 3) * 32;
+    umma_bf16_ss(d, umma_sdesc_sw128(qa + off, 16, 1024), umma_sdesc_sw128(kb + off, 16, 1024),
+                 idesc, k > 0);
+  }
+}
+
+// O (+)= P V_j (M = 128 rows, N = 128 head dims, K = 128 keys): P K-major
+// from `pa`, V MN-major (its head dim contiguous): 16 keys = two 8-row
+// swizzle groups = 2 KiB per step, the two 64-dim halves 16 KiB apart.
+__device__ __forceinline__ void pf_issue_pv(uint32_t pa, uint32_t vb, uint32_t tmem, bool first) {
+  constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfD, true);
+#pragma unroll
+  for (int k = 0; k < kPfKeys / 16; ++k) {
+    const uint32_t aoff = (k >> 2) * kPfHalfBytes + (k & 3) * 32;
+    umma_bf16_ss(tmem + kPfColO, umma_sdesc_sw128(pa + aoff, 16, 1024),
+                 umma_sdesc_sw128(vb + k * 2048, kPfHalfBytes, 1024), idesc,
+                 (first && k == 0) ? 0u : 1u);
+  }
+}
+
+// Warp 5, one thread.  Issue order: S_0, S_1, then per tile j: PV_j (once
+// P_j is written), S_{j+2} (once the softmax has read S_j out of its
+// buffer).  Each group's completion is signalled with tcgen05.commit.
+__device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem, int nt, bool hilo,
+                                       unsigned long long tmo) {
+  if (pf_wait(sb, sb.q_full, 0, tmo)) {
+    tc_fence_after_sync();
+    bool ok = true;
+    for (int j = 0; j < 2 && j < nt && ok; ++j) {
+      ok = pf_wait(sb, sb.k_full[j], 0, tmo);
+      if (!ok) break;
+      tc_fence_after_sync();
+      pf_issue_qk(smem, tmem, j);
+      umma_commit(bar_addr(sb.s_full[j]));
+      umma_commit(bar_addr(sb.k_empty[j]));
+    }
+    for (int j = 0; j < nt && ok; ++j) {
+      const int s = j & 1;
+      const uint32_t par = (j >> 1) & 1;
+      if (!pf_wait(sb, sb.p_full[s], par, tmo) || !pf_wait(sb, sb.v_full[s], par, tmo)) break;
+      tc_fence_after_sync();
+      const uint32_t vb = smem + kPfSmemV + s * kPfTileBytes;
+      pf_issue_pv(smem + kPfSmemP + s * kPfTileBytes, vb, tmem, j == 0);
+      if (hilo) pf_issue_pv(smem + kPfSmemQ, vb, tmem, false);   // the lo parts of P
+      umma_commit(bar_addr(sb.pv_done[s]));
+      umma_commit(bar_addr(sb.v_empty[s]));
+      if (j + 2 < nt) {
+        if (!pf_wait(sb, sb.s_free[s], par, tmo) || !pf_wait(sb, sb.k_full[s], par ^ 1, tmo)) break;
+        tc_fence_after_sync();
+        pf_issue_qk(smem, tmem, j + 2);
+        umma_commit(bar_addr(sb.s_full[s]));
+        umma_commit(bar_addr(sb.k_empty[s]));
+      }
+    }
+  }
+  // Nothing issued may still run when TMEM is freed.
+  umma_commit(bar_addr(sb.drain));
+  if (!mbar_wait_bounded(bar_addr(sb.drain), 0, tmo)) raise_status(kStatusTimeout);
+}
+
+// Reads 128 fp32 columns of this thread's TMEM lane into v (four loads in
+// flight, one wait).
+__device__ __forceinline__ void pf_ld_row(uint32_t taddr, uint32_t (&v)[4][32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
+  tmem_wait_ld();
+}
+
+// Multiplies this thread's O row (TMEM) by f, 32 columns at a time.
+__device__ __forceinline__ void pf_rescale_o(uint32_t trow, float f) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld32(trow + kPfColO + c * 32, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+    tmem_st32(trow + kPfColO + c * 32, o);
+  }
+  tmem_wait_st();
+}
+
+// Warps 0-3: thread r owns query row r of the tile (TMEM lane r).  Per KV
+// tile j: read S_j, mask (the diagonal tile keeps keys c <= r), update the
+// row's reference max m (base 2, kept unless the tile's max exceeds it by
+// more than 2^8: then O and the denominator are rescaled), write
+// P = 2^(s*scale*log2e - m) as bf16 into the K-major swizzled P buffer
+// (plus its lo part into the spent Q buffer for q-tile 0), and accumulate
+// the fp32 denominator.  Finally O / l is stored for the rows that exist.
+__device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t tmem, int warp,
+                                           int lane, int nt, bool hilo, const PrefillArgs& a,
+                                           long long out_row0, int rows_valid, int h,
+                                           unsigned long long tmo) {
+  const int r = warp * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const float sl2 = a.scale_log2;
+  float m_used = -INFINITY, l = 0.f;
+  bool ok = true;
+  for (int j = 0; j < nt; ++j) {
+    const int s = j & 1;
+    const uint32_t par = (j >> 1) & 1;
+    if (!(ok = pf_wait_warp(sb, sb.s_full[s], par, tmo))) break;
+    tc_fence_after_sync();
+    uint32_t v[4][32];
+    pf_ld_row(trow + (s ? kPfColS1 : kPfColS0), v);
+    tc_fence_before_sync();
+    mbar_arrive(bar_addr(sb.s_free[s]));
+
+    const bool diag = (j == nt - 1);
+    // tile max (or min, for a negative scale) over the row's valid keys
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float mn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      const float x = __uint_as_float(v[c >> 5][c & 31]);
+      const bool valid = !diag || c <= r;
+      mx[c & 3] = fmaxf(mx[c & 3], valid ? x : -INFINITY);
+      if (sl2 < 0.f) mn[c & 3] = fminf(mn[c & 3], valid ? x : INFINITY);
+    }
+    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    const float tmin = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+    const float mt = sl2 > 0.f ? tmax * sl2 : (sl2 < 0.f ? tmin * sl2 : 0.f);
+    const float m_new = fmaxf(m_used, mt);
+    const bool resc = m_new > m_used + kPfRescaleLog2;   // always true on the first tile
+    float factor = 1.f;
+    if (resc) {
+      factor = ex2_approx(m_used - m_new);                 // 0 on the first tile
+      l *= factor;
+      m_used = m_new;
+    }
+    // P buffer s is free once PV_{j-2} has completed; O may be rescaled once
+    // PV_{j-1} has.
+    if (j >= 2 && !(ok = pf_wait_warp(sb, sb.pv_done[s], ((j - 2) >> 1) & 1, tmo))) break;
+    if (j >= 1 && __any_sync(kFull, resc)) {
+      if (!(ok = pf_wait_warp(sb, sb.pv_done[s ^ 1], ((j - 1) >> 1) & 1, tmo))) break;
+      tc_fence_after_sync();
+      pf_rescale_o(trow, factor);
+    }
+
+    const float neg = -m_used;
+    const uint32_t pb = smem + kPfSmemP + s * kPfTileBytes + r * 128;
+    const uint32_t lb = smem + kPfSmemQ + r * 128;
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c8 = 0; c8 < 16; ++c8) {
+      float p[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int c = c8 * 8 + e;
+        const bool valid = !diag || c <= r;
+        p[e] = valid ? ex2_approx(fmaf(__uint_as_float(v[c >> 5][c & 31]), sl2, neg)) : 0.f;
+        ls[e & 3] += p[e];
+      }
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
+      const uint32_t off = (c8 >> 3) * kPfHalfBytes + ((uint32_t)((c8 & 7) ^ (r & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + off), "r"(w[0]),
+                   "r"(w[1]), "r"(w[2]), "r"(w[3])
+                   : "memory");
+      if (hilo) {
+        uint32_t z[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          z[e] = pack_bf16x2(p[2 * e] - bf16lo_to_f32(w[e]), p[2 * e + 1] - bf16hi_to_f32(w[e]));
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lb + off), "r"(z[0]),
+                     "r"(z[1]), "r"(z[2]), "r"(z[3])
+                     : "memory");
+      }
+    }
+    l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+    fence_proxy_async_smem();   // generic-proxy P writes -> tensor-core reads
+    tc_fence_before_sync();
+    mbar_arrive(bar_addr(sb.p_full[s]));
+  }
+  if (!ok) return;
+
+  // Epilogue: O / l for the rows of this tile that exist.
+  if (!pf_wait_warp(sb, sb.pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, tmo)) return;
+  tc_fence_after_sync();
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float* dst = a.out + ((out_row0 + r) * a.h_q + h) * (long long)kPfD;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld32(trow + kPfColO + c * 32, o);
+    tmem_wait_ld();
+    if (r < rows_valid) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 val = make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                                       __uint_as_float(o[e + 2]) * inv,
+                                       __uint_as_float(o[e + 3]) * inv);
+        *reinterpret_cast<float4*>(dst + c * 32 + e) = val;
+      }
+    }
+  }
+}
+
+// Grid (h_q, B, n_qtiles): block (h, b, z) takes q-tile t = n_qtiles-1-z of
+// head h of sequence b, so the longest rows (most KV tiles) start first and
+// the heads of one kv group run side by side (their K/V tiles shared in L2).
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_tc_bf16(const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
+  __shared__ PfBars sb;
+  extern __shared__ uint8_t pf_dyn[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int t = a.n_qtiles - 1 - (int)blockIdx.z;
+
+  grid_dependency_wait();
+  // Sequence b: first row (prefix sum of the non-negative lengths) and length.
+  long long off = 0;
+  for (int i = lane; i < b; i += 32) {
+    const int v = a.seqlens[i];
+    off += v > 0 ? v : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(kFull, off, o);
+  const int Sraw = a.seqlens[b];
+  long long S = Sraw > 0 ? Sraw : 0;
+  if (threadIdx.x == 0 && h == 0 && t == 0) {
+    if (Sraw < 0) raise_status(kStatusNegSeqlen);
+    if (S > (long long)a.n_qtiles * kPfRows || off + S > a.total_rows)
+      raise_status(kStatusSeqlenOverMax);
+  }
+  if (off + S > a.total_rows) S = a.total_rows > off ? a.total_rows - off : 0;
+  if ((long long)t * kPfRows >= S) return;   // the whole CTA: no rows here
+  allow_dependent_launch();
+
+  const int nt = t + 1;
+  const bool hilo = (t == 0);
+  const long long qrow = off + (long long)t * kPfRows;
+  const int rows_valid = (int)(S - (long long)t * kPfRows < kPfRows ? S - (long long)t * kPfRows
+                                                                     : kPfRows);
+  const uint32_t smem = (smem_u32(pf_dyn) + 1023u) & ~1023u;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_addr(sb.q_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_addr(sb.k_full[s]), 1);
+      mbar_init(bar_addr(sb.k_empty[s]), 1);
+      mbar_init(bar_addr(sb.v_full[s]), 1);
+      mbar_init(bar_addr(sb.v_empty[s]), 1);
+      mbar_init(bar_addr(sb.s_full[s]), 1);
+      mbar_init(bar_addr(sb.s_free[s]), 4 * 32);
+      mbar_init(bar_addr(sb.p_full[s]), 4 * 32);
+      mbar_init(bar_addr(sb.pv_done[s]), 1);
+    }
+    mbar_init(bar_addr(sb.drain), 1);
+    sb.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&qmap);
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  if (warp == 5) tmem_alloc(smem_u32(&sb.tmem_base), kPfTmemCols);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = sb.tmem_base;
+
+  if (warp < 4) {
+    pf_softmax(sb, smem, tmem, warp, lane, nt, hilo, a, qrow, rows_valid, h, a.timeout_ns);
+  } else if (warp == 4) {
+    if (lane == 0)
+      pf_producer(sb, smem, &qmap, &kmap, &vmap, h, h / a.G, qrow, off, nt, a.timeout_ns);
+  } else {
+    if (lane == 0) pf_mma(sb, smem, tmem, nt, hilo, a.timeout_ns);
+  }
+  __syncwarp();
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kPfTmemCols);
+  }
+}
+
+}  // namespace gqa

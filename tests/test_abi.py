@@ -9,7 +9,8 @@ import pytest
 import importlib.util
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gqa_decode.h")
+INCLUDE = os.path.join(ROOT, "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
 
 OK, INVALID, UNSUPPORTED, CUDA_ERR, WORKSPACE = 0, 1, 2, 3, 4
 
@@ -31,6 +32,7 @@ def lib():
     lib.gqa_decode_attn_chunked.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
     lib.gqa_decode_partial.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
     lib.mlo_merge.argtypes = [vp, vp, vp, vp, ci, ci, ci, vp]
+    lib.gqa_prefill_attn.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
     lib.gqa_decode_workspace_size.restype = sz
     lib.gqa_decode_workspace_size.argtypes = [ci] * 5
     lib.gqa_decode_chunked_workspace_size.restype = sz
@@ -40,14 +42,16 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return re.findall(r"GQA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    names = []
+    for h in HEADERS:
+        names += re.findall(r"GQA_API\s+[\w\s\*]+?\b(\w+)\s*\(", open(h).read())
+    return names
 
 
 def test_header_declares_the_path():
     names = set(declared_functions())
     for required in ["gqa_decode_attn", "gqa_decode_partial", "mlo_merge", "gqa_decode_attn_chunked",
-                     "gqa_decode_get_status", "gqa_decode_workspace_size"]:
+                     "gqa_decode_get_status", "gqa_decode_workspace_size", "gqa_prefill_attn"]:
         assert required in names
 
 
@@ -55,7 +59,7 @@ def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
     assert len(names) >= 10
     for n in names:
-        assert hasattr(lib, n), f"{n} declared in gqa_decode.h but not exported"
+        assert hasattr(lib, n), f"{n} declared in a header but not exported"
 
 
 def test_version_and_error_strings(lib):
@@ -134,3 +138,30 @@ def test_launch_count_query_without_a_gpu(lib):
     assert lib.gqa_decode_launches_per_call(0, 8, 2, 128, 4, 1) == 0      # empty batch
     assert lib.gqa_decode_launches_per_call(2, 8, 2, 128, 4, 0) == 1      # fp32: one kernel
     assert lib.gqa_decode_launches_per_call(2, 6, 4, 128, 4, 1) == -INVALID
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(h_q=6, h_kv=4), INVALID),
+    (dict(d=64), UNSUPPORTED),               # prefill runs d_head = 128 only
+    (dict(d=0), INVALID),
+    (dict(dtype=0), UNSUPPORTED),            # fp32 prefill is not provided
+    (dict(dtype=7), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(rows=-1), INVALID),
+    (dict(max_seqlen=-1), INVALID),
+    (dict(max_seqlen=0), INVALID),           # rows exist, so some sequence is longer
+    (dict(max_seqlen=128 * 65536), UNSUPPORTED),
+    (dict(q=0), INVALID),
+    (dict(v=FAKE + 8), INVALID),             # misaligned
+    (dict(out=FAKE + 4), INVALID),
+    (dict(B=0), OK),                         # nothing to do
+    (dict(rows=0), OK),
+])
+def test_prefill_argument_checks(lib, kw, expect):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, out=FAKE, B=2, rows=300, max_seqlen=200, h_q=8, h_kv=2,
+             d=128, scale=0.1, dtype=1)
+    a.update(kw)
+    rc = lib.gqa_prefill_attn(a["q"], a["k"], a["v"], a["sl"], a["out"], a["B"], a["rows"],
+                              a["max_seqlen"], a["h_q"], a["h_kv"], a["d"], a["scale"], a["dtype"], None)
+    assert rc == expect

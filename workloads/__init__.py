@@ -180,3 +180,69 @@ def random_case(B, h_q, h_kv, d, seqlens, dtype="bf16", seed=0, std=1.0, scale=N
                  scale=(1 / math.sqrt(d)) if scale is None else scale, n_splits=n_splits,
                  chunk_len=chunk_len, std=std)
     return generate(cfg, seed=seed, seqlens=list(seqlens))
+
+
+# ---------------------------------------------------------------- prefill
+
+@dataclass
+class PrefillWorkload:
+    """Causal prefill inputs: q [rows, h_q, d], k, v [rows, h_kv, d], packed by
+    sequence (sequence b occupies rows S_0 + ... + S_{b-1} onwards)."""
+    name: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    seqlens: torch.Tensor
+    h_q: int
+    h_kv: int
+    d: int
+    scale: float
+
+    @property
+    def max_seqlen(self) -> int:
+        return int(self.seqlens.max()) if self.seqlens.numel() else 0
+
+    @property
+    def flops(self) -> int:
+        """Multiply-adds x 2 of the attended (query, key) pairs only: QK^T and
+        PV, each 2 * d per pair per query head; pairs = S_b (S_b + 1) / 2."""
+        pairs = sum(int(s) * (int(s) + 1) // 2 for s in self.seqlens.tolist())
+        return 4 * self.d * self.h_q * pairs
+
+
+# Llama-2 70B attention shape (64 query / 8 kv heads of 128) at the 2k
+# prefill length of the tt-metal "[Llama2] Perf burndown" page; a ragged
+# batch of the same shape.  Seeds 2000 + index.
+PREFILL_CONFIGS = {
+    "llama70b_prefill2k": dict(index=1, B=1, S=2048, S_min=0, h_q=64, h_kv=8, d=128),
+    "prefill_ragged": dict(index=2, B=16, S=4096, S_min=1, h_q=64, h_kv=8, d=128),
+}
+
+
+def prefill_case(seqlens, h_q, h_kv, d, dtype="bf16", seed=0, std=1.0, scale=None,
+                 name="case") -> PrefillWorkload:
+    """N(0, std^2) causal-prefill inputs with explicit lengths.  Draws q, then
+    k, then v (PCG64 ``seed``, fp32 chunks, rounded once to ``dtype``)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    sl = torch.as_tensor(np.asarray(list(seqlens), dtype=np.int32))
+    rows = int(sl.sum())
+    dt = _torch_dtype(dtype)
+    q = _normal(rng, (rows, h_q, d), std, dt)
+    k = _normal(rng, (rows, h_kv, d), std, dt)
+    v = _normal(rng, (rows, h_kv, d), std, dt)
+    return PrefillWorkload(name, q, k, v, sl, h_q, h_kv, d,
+                           (1 / math.sqrt(d)) if scale is None else float(scale))
+
+
+def generate_prefill(name: str) -> PrefillWorkload:
+    """The seeded prefill workload ``name``: lengths (ragged: uniform integers
+    in [S_min, S] drawn first from seed 2000 + index), then q, k, v."""
+    c = PREFILL_CONFIGS[name]
+    seed = 2000 + c["index"]
+    if c["S_min"] > 0:
+        rng = np.random.Generator(np.random.PCG64(seed))
+        sl = rng.integers(c["S_min"], c["S"], size=c["B"], endpoint=True).tolist()
+        seed += 100
+    else:
+        sl = [c["S"]] * c["B"]
+    return prefill_case(sl, c["h_q"], c["h_kv"], c["d"], seed=seed, name=name)
