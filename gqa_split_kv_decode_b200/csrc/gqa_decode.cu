@@ -522,16 +522,16 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
 // ------------------------------------------------------------ prefill
 
 // 3-D view (d = 128, head, row) of a packed bf16 [rows][heads][128] tensor;
-// box = 64 d x 1 head x 128 rows, 128-byte swizzle.  The row extent is the
-// tensor's own, so a tile that runs past the last row reads zeros.
-bool encode_rows_map(CUtensorMap* map, const void* base, int heads, int rows) {
+// box = 64 d x 1 head x box_rows rows, 128-byte swizzle.  The row extent is
+// the tensor's own, so a tile that runs past the last row reads zeros.
+bool encode_rows_map(CUtensorMap* map, const void* base, int heads, int rows, int box_rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kPfD), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kPfD) * 2,
                                  static_cast<cuuint64_t>(heads) * kPfD * 2};
-  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kPfRows)};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -560,8 +560,9 @@ int prefill(const void* q, const void* k, const void* v, const int32_t* seqlens,
   static std::atomic<uint64_t> attr_done{0};
   if (int rc = ensure_smem_attr(prefill_tc_bf16, kPfDynSmem, attr_done)) return rc;
   CUtensorMap qmap, kmap, vmap;
-  if (!encode_rows_map(&qmap, q, h_q, total_rows) || !encode_rows_map(&kmap, k, h_kv, total_rows) ||
-      !encode_rows_map(&vmap, v, h_kv, total_rows))
+  if (!encode_rows_map(&qmap, q, h_q, total_rows, kPfRows) ||
+      !encode_rows_map(&kmap, k, h_kv, total_rows, kPfKeys) ||
+      !encode_rows_map(&vmap, v, h_kv, total_rows, kPfKeys))
     return GQA_ERR_CUDA;
   PrefillArgs a{};
   a.seqlens = seqlens;

@@ -8,22 +8,28 @@
 //   O_i = sum_{j<=i} e^{s_ij - m_i} v_j / sum_{j<=i} e^{s_ij - m_i},
 //   s_ij = scale <q_i, k_j>,  query head h reading kv head h / (h_q / h_kv).
 //
-// One CTA = 128 query rows of one head of one sequence.  Six warps:
+// One CTA = 128 query rows of one head of one sequence; two CTAs share an
+// SM, so one's tensor-core work fills the other's softmax time.  Six warps:
 //   warps 0-3  softmax: thread r owns row r (TMEM lane r) -- reads S from
-//              TMEM, keeps the row's running max and denominator, writes P
-//              (bf16) to shared memory, rescales O in TMEM when needed, and
-//              finally normalises O and stores it;
-//   warp 4     TMA producer: Q once, then K and V tiles of 128 keys through
+//              TMEM, keeps the row's reference max and denominator, writes P
+//              back into TMEM over the S it came from, rescales O when the
+//              max moves, and finally normalises O and stores it;
+//   warp 4     TMA producer: Q once, then 64-key K and V tiles through
 //              two-stage rings;
-//   warp 5     MMA issuer (one thread): S = Q K^T into one of two TMEM S
-//              buffers, then O += P V into the TMEM O accumulator.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384) of a 512-column
-// allocation (fp32, lane = query row).
+//   warp 5     MMA issuer (one thread): S_j = Q K_j^T from shared memory
+//              into one of two TMEM S buffers, then O += P_j V_j with P read
+//              from TMEM.
+// TMEM (256 columns, fp32, lane = query row): S0 [0,64), S1 [64,128),
+// O [128,256).  P_j replaces S_j in place: keys 32c..32c+31 of the tile
+// (S columns [32c, 32c+32)) become their bf16 hi parts in columns
+// [32c, 32c+16) and lo parts (p - hi, rounded) in [32c+16, 32c+32).
 //
-// Rows whose whole key range is short (the first 128 positions of a
-// sequence, q-tile 0) take P as two bf16 parts, hi + lo, summed by two MMAs
-// into O, so a row of a few keys keeps near-fp32 weights; longer rows use
-// one bf16 P (its rounding averages out over the keys).
+// Precision: the P V product normally takes the hi parts only (one bf16 P).
+// A (128-row, 64-key) block also adds the lo parts -- so its P is exact to
+// ~2^-17 -- whenever some row's tile mass exceeds a quarter of that row's
+// running denominator; that covers every short row and every tile that
+// carries a row's dominant keys, where a single bf16 rounding of the
+// weights would show in the output.
 #pragma once
 
 #include "device_common.cuh"
@@ -31,22 +37,24 @@
 
 namespace gqa {
 
-constexpr int kPfRows = 128;      // query rows per CTA (MMA M)
-constexpr int kPfKeys = 128;      // keys per K/V tile (MMA N of QK^T, K of PV)
-constexpr int kPfD = 128;         // head dim (MMA K of QK^T, N of PV)
+constexpr int kPfRows = 128;                   // query rows per CTA (MMA M)
+constexpr int kPfKeys = 64;                    // keys per K/V tile
+constexpr int kPfD = 128;                      // head dim
 constexpr int kPfThreads = 192;
-constexpr int kPfHalfBytes = kPfRows * 128;        // one 64-column half of a 128-row tile
-constexpr int kPfTileBytes = 2 * kPfHalfBytes;     // 32 KiB
-// Shared memory: Q, K[2], V[2], P[2] tiles, 1024-byte aligned.
+constexpr int kPfQHalf = kPfRows * 128;        // 64 dims x 128 rows: 16 KiB
+constexpr int kPfKvHalf = kPfKeys * 128;       // 64 dims x 64 keys: 8 KiB
+constexpr int kPfQBytes = 2 * kPfQHalf;        // 32 KiB
+constexpr int kPfKvBytes = 2 * kPfKvHalf;      // 16 KiB
+// Shared memory: Q, K[2], V[2], 1024-byte aligned.
 constexpr int kPfSmemQ = 0;
-constexpr int kPfSmemK = kPfSmemQ + kPfTileBytes;
-constexpr int kPfSmemV = kPfSmemK + 2 * kPfTileBytes;
-constexpr int kPfSmemP = kPfSmemV + 2 * kPfTileBytes;
-constexpr int kPfSmemBytes = kPfSmemP + 2 * kPfTileBytes;   // 224 KiB
-constexpr int kPfDynSmem = kPfSmemBytes + 1024;            // + alignment slack
-constexpr uint32_t kPfTmemCols = 512;
-constexpr uint32_t kPfColS0 = 0, kPfColS1 = 128, kPfColO = 256;
+constexpr int kPfSmemK = kPfSmemQ + kPfQBytes;
+constexpr int kPfSmemV = kPfSmemK + 2 * kPfKvBytes;
+constexpr int kPfSmemBytes = kPfSmemV + 2 * kPfKvBytes;   // 96 KiB
+constexpr int kPfDynSmem = kPfSmemBytes + 1024;          // + alignment slack
+constexpr uint32_t kPfTmemCols = 256;
+constexpr uint32_t kPfColO = 128;
 constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale: keep the max unless it grew by > 2^8
+constexpr float kPfLoShare = 0.25f;     // a tile above this share of a row's mass takes lo parts
 
 struct PrefillArgs {
   const int32_t* seqlens;   // [B] device
@@ -58,14 +66,14 @@ struct PrefillArgs {
   unsigned long long timeout_ns;
 };
 
-// Barriers of one CTA (shared memory).
+// Barriers and flags of one CTA (shared memory).
 struct PfBars {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t drain;
+  int lo_tile[2];           // j + 1 when tile j's block needs the lo parts
   uint32_t tmem_base;
   int abort;
 };
@@ -91,13 +99,14 @@ __device__ __forceinline__ bool pf_wait_warp(PfBars& sb, uint64_t& bar, uint32_t
   return __all_sync(kFull, ok);
 }
 
-// Loads a 128-row x 128-column bf16 tile as two 64-column boxes (128-byte
-// swizzle): columns [0,64) at dst, [64,128) at dst + 16 KiB.
-__device__ __forceinline__ void pf_load_tile(uint32_t dst, const CUtensorMap* map, int head,
-                                             long long row, uint32_t bar, uint64_t policy) {
-  mbar_arrive_expect_tx(bar, kPfTileBytes);
+// Loads a rows x 128-dim bf16 tile as two 64-dim boxes (128-byte swizzle):
+// dims [0,64) at dst, [64,128) at dst + half_bytes.
+__device__ __forceinline__ void pf_load_tile(uint32_t dst, uint32_t half_bytes,
+                                             const CUtensorMap* map, int head, long long row,
+                                             uint32_t bar, uint64_t policy) {
+  mbar_arrive_expect_tx(bar, 2 * half_bytes);
   tma_load_3d(dst, map, 0, head, (int)row, bar, policy);
-  tma_load_3d(dst + kPfHalfBytes, map, 64, head, (int)row, bar, policy);
+  tma_load_3d(dst + half_bytes, map, 64, head, (int)row, bar, policy);
 }
 
 // Warp 4, one thread: Q, then K_j / V_j for j = 0 .. nt-1 through the rings.
@@ -110,24 +119,26 @@ __device__ __forceinline__ void pf_producer(PfBars& sb, uint32_t smem, const CUt
                                             unsigned long long tmo) {
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  pf_load_tile(smem + kPfSmemQ, qmap, h, qrow, bar_addr(sb.q_full), pol_q);
+  pf_load_tile(smem + kPfSmemQ, kPfQHalf, qmap, h, qrow, bar_addr(sb.q_full), pol_q);
   int issued = 0;
   for (int j = 0; j < nt; ++j) {
     const int s = j & 1;
     const uint32_t par = ((j >> 1) - 1) & 1;
     const long long row = krow0 + (long long)j * kPfKeys;
     if (j >= 2 && !pf_wait(sb, sb.k_empty[s], par, tmo)) break;
-    pf_load_tile(smem + kPfSmemK + s * kPfTileBytes, kmap, g, row, bar_addr(sb.k_full[s]), pol_kv);
+    pf_load_tile(smem + kPfSmemK + s * kPfKvBytes, kPfKvHalf, kmap, g, row,
+                 bar_addr(sb.k_full[s]), pol_kv);
     if (j >= 2 && !pf_wait(sb, sb.v_empty[s], par, tmo)) {
       issued = 2 * j + 1;
       break;
     }
-    pf_load_tile(smem + kPfSmemV + s * kPfTileBytes, vmap, g, row, bar_addr(sb.v_full[s]), pol_kv);
+    pf_load_tile(smem + kPfSmemV + s * kPfKvBytes, kPfKvHalf, vmap, g, row,
+                 bar_addr(sb.v_full[s]), pol_kv);
     issued = 2 * j + 2;
   }
   // Drain: the last K and V load of each stage (earlier ones are implied,
   // since a stage is refilled only after its previous load was consumed).
-  mbar_wait_bounded(bar_addr(sb.q_full), 0, tmo);
+  if (!mbar_wait_bounded(bar_addr(sb.q_full), 0, tmo)) raise_status(kStatusTimeout);
   for (int n = issued - 1; n >= 0 && n >= issued - 4; --n) {
     const int j = n >> 1;
     uint64_t& bar = (n & 1) ? sb.v_full[j & 1] : sb.k_full[j & 1];
@@ -135,40 +146,42 @@ __device__ __forceinline__ void pf_producer(PfBars& sb, uint32_t smem, const CUt
   }
 }
 
-// S_j = Q K_j^T (M = 128 rows, N = 128 keys, K = 128 head dims): eight
-// K = 16 steps; both operands K-major, each step 32 bytes further along the
-// swizzled 128-byte rows, the second 64 dims in the tile's second half.
+// S_j = Q K_j^T (M = 128 rows, N = 64 keys, K = 128 dims): eight K = 16
+// steps, both operands K-major, each step 32 bytes further along the
+// swizzled 128-byte rows, dims 64..127 in each tile's second half.
 __device__ __forceinline__ void pf_issue_qk(uint32_t smem, uint32_t tmem, int j) {
   constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfKeys, false);
   const uint32_t qa = smem + kPfSmemQ;
-  const uint32_t kb = smem + kPfSmemK + (j & 1) * kPfTileBytes;
-  const uint32_t d = tmem + ((j & 1) ? kPfColS1 : kPfColS0);
+  const uint32_t kb = smem + kPfSmemK + (j & 1) * kPfKvBytes;
+  const uint32_t d = tmem + (j & 1) * kPfKeys;
 #pragma unroll
   for (int k = 0; k < kPfD / 16; ++k) {
-    const uint32_t off = (k >> 2) * kPfHalfBytes + (k & 3) * 32;
-    umma_bf16_ss(d, umma_sdesc_sw128(qa + off, 16, 1024), umma_sdesc_sw128(kb + off, 16, 1024),
-                 idesc, k > 0);
+    const uint32_t sub = (k & 3) * 32;
+    umma_bf16_ss(d, umma_sdesc_sw128(qa + (k >> 2) * kPfQHalf + sub, 16, 1024),
+                 umma_sdesc_sw128(kb + (k >> 2) * kPfKvHalf + sub, 16, 1024), idesc, k > 0);
   }
 }
 
-// O (+)= P V_j (M = 128 rows, N = 128 head dims, K = 128 keys): P K-major
-// from `pa`, V MN-major (its head dim contiguous): 16 keys = two 8-row
-// swizzle groups = 2 KiB per step, the two 64-dim halves 16 KiB apart.
-__device__ __forceinline__ void pf_issue_pv(uint32_t pa, uint32_t vb, uint32_t tmem, bool first) {
+// O (+)= P V_j (M = 128 rows, N = 128 dims, K = 64 keys): P from TMEM (the
+// hi or lo columns of each 32-key chunk), V MN-major (its dims contiguous):
+// 16 keys = two 8-row swizzle groups = 2 KiB per step, the two 64-dim halves
+// 8 KiB apart.
+__device__ __forceinline__ void pf_issue_pv(uint32_t tmem, int j, uint32_t vb, bool lo,
+                                            bool overwrite) {
   constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfD, true);
+  const uint32_t p = tmem + (j & 1) * kPfKeys + (lo ? 16 : 0);
 #pragma unroll
   for (int k = 0; k < kPfKeys / 16; ++k) {
-    const uint32_t aoff = (k >> 2) * kPfHalfBytes + (k & 3) * 32;
-    umma_bf16_ss(tmem + kPfColO, umma_sdesc_sw128(pa + aoff, 16, 1024),
-                 umma_sdesc_sw128(vb + k * 2048, kPfHalfBytes, 1024), idesc,
-                 (first && k == 0) ? 0u : 1u);
+    umma_bf16_ts(tmem + kPfColO, p + (k >> 1) * 32 + (k & 1) * 8,
+                 umma_sdesc_sw128(vb + k * 2048, kPfKvHalf, 1024), idesc,
+                 (overwrite && k == 0) ? 0u : 1u);
   }
 }
 
-// Warp 5, one thread.  Issue order: S_0, S_1, then per tile j: PV_j (once
-// P_j is written), S_{j+2} (once the softmax has read S_j out of its
-// buffer).  Each group's completion is signalled with tcgen05.commit.
-__device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem, int nt, bool hilo,
+// Warp 5, one thread.  Issue order: S_0, S_1, then per tile j: PV_j (once P_j
+// is in TMEM; with the lo parts when the softmax asked for them), then
+// S_{j+2} into the same S buffer once PV_j has finished reading P_j there.
+__device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem, int nt,
                                        unsigned long long tmo) {
   if (pf_wait(sb, sb.q_full, 0, tmo)) {
     tc_fence_after_sync();
@@ -186,13 +199,15 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
       const uint32_t par = (j >> 1) & 1;
       if (!pf_wait(sb, sb.p_full[s], par, tmo) || !pf_wait(sb, sb.v_full[s], par, tmo)) break;
       tc_fence_after_sync();
-      const uint32_t vb = smem + kPfSmemV + s * kPfTileBytes;
-      pf_issue_pv(smem + kPfSmemP + s * kPfTileBytes, vb, tmem, j == 0);
-      if (hilo) pf_issue_pv(smem + kPfSmemQ, vb, tmem, false);   // the lo parts of P
+      const uint32_t vb = smem + kPfSmemV + s * kPfKvBytes;
+      pf_issue_pv(tmem, j, vb, false, j == 0);
+      if (*reinterpret_cast<volatile int*>(&sb.lo_tile[s]) == j + 1)
+        pf_issue_pv(tmem, j, vb, true, false);
       umma_commit(bar_addr(sb.pv_done[s]));
       umma_commit(bar_addr(sb.v_empty[s]));
       if (j + 2 < nt) {
-        if (!pf_wait(sb, sb.s_free[s], par, tmo) || !pf_wait(sb, sb.k_full[s], par ^ 1, tmo)) break;
+        if (!pf_wait(sb, sb.pv_done[s], par, tmo) || !pf_wait(sb, sb.k_full[s], par ^ 1, tmo))
+          break;
         tc_fence_after_sync();
         pf_issue_qk(smem, tmem, j + 2);
         umma_commit(bar_addr(sb.s_full[s]));
@@ -203,14 +218,6 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
   // Nothing issued may still run when TMEM is freed.
   umma_commit(bar_addr(sb.drain));
   if (!mbar_wait_bounded(bar_addr(sb.drain), 0, tmo)) raise_status(kStatusTimeout);
-}
-
-// Reads 128 fp32 columns of this thread's TMEM lane into v (four loads in
-// flight, one wait).
-__device__ __forceinline__ void pf_ld_row(uint32_t taddr, uint32_t (&v)[4][32]) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
-  tmem_wait_ld();
 }
 
 // Multiplies this thread's O row (TMEM) by f, 32 columns at a time.
@@ -227,17 +234,17 @@ __device__ __forceinline__ void pf_rescale_o(uint32_t trow, float f) {
   tmem_wait_st();
 }
 
-// Warps 0-3: thread r owns query row r of the tile (TMEM lane r).  Per KV
-// tile j: read S_j, mask (the diagonal tile keeps keys c <= r), update the
-// row's reference max m (base 2, kept unless the tile's max exceeds it by
-// more than 2^8: then O and the denominator are rescaled), write
-// P = 2^(s*scale*log2e - m) as bf16 into the K-major swizzled P buffer
-// (plus its lo part into the spent Q buffer for q-tile 0), and accumulate
-// the fp32 denominator.  Finally O / l is stored for the rows that exist.
-__device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t tmem, int warp,
-                                           int lane, int nt, bool hilo, const PrefillArgs& a,
-                                           long long out_row0, int rows_valid, int h,
-                                           unsigned long long tmo) {
+// Warps 0-3: thread r owns query row r of the tile (TMEM lane r).  Per K/V
+// tile j: read S_j, mask (key c of the tile is valid while
+// c <= r + 128 t - 64 j), update the row's reference max m (base 2, kept
+// unless the tile's max exceeds it by more than 2^8: then O and the
+// denominator are rescaled), write P = 2^(s * scale * log2e - m) into TMEM
+// as bf16 hi and lo parts, accumulate the fp32 denominator, and flag the
+// block for the lo MMA when this tile holds more than a quarter of the row's
+// mass so far.  Finally O / l is stored for the rows that exist.
+__device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, int lane, int t,
+                                           int nt, const PrefillArgs& a, long long out_row0,
+                                           int rows_valid, int h, unsigned long long tmo) {
   const int r = warp * 32 + lane;
   const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   const float sl2 = a.scale_log2;
@@ -245,22 +252,21 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
   bool ok = true;
   for (int j = 0; j < nt; ++j) {
     const int s = j & 1;
-    const uint32_t par = (j >> 1) & 1;
-    if (!(ok = pf_wait_warp(sb, sb.s_full[s], par, tmo))) break;
+    if (!(ok = pf_wait_warp(sb, sb.s_full[s], (j >> 1) & 1, tmo))) break;
     tc_fence_after_sync();
-    uint32_t v[4][32];
-    pf_ld_row(trow + (s ? kPfColS1 : kPfColS0), v);
-    tc_fence_before_sync();
-    mbar_arrive(bar_addr(sb.s_free[s]));
+    const uint32_t sbuf = trow + s * kPfKeys;
+    uint32_t v[2][32];
+    tmem_ld32(sbuf, v[0]);
+    tmem_ld32(sbuf + 32, v[1]);
+    tmem_wait_ld();
 
-    const bool diag = (j == nt - 1);
-    // tile max (or min, for a negative scale) over the row's valid keys
+    const int lim = r + kPfRows * t - kPfKeys * j;   // keys c <= lim are causal
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     float mn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
 #pragma unroll
-    for (int c = 0; c < 128; ++c) {
+    for (int c = 0; c < kPfKeys; ++c) {
       const float x = __uint_as_float(v[c >> 5][c & 31]);
-      const bool valid = !diag || c <= r;
+      const bool valid = c <= lim;
       mx[c & 3] = fmaxf(mx[c & 3], valid ? x : -INFINITY);
       if (sl2 < 0.f) mn[c & 3] = fminf(mn[c & 3], valid ? x : INFINITY);
     }
@@ -275,9 +281,7 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
       l *= factor;
       m_used = m_new;
     }
-    // P buffer s is free once PV_{j-2} has completed; O may be rescaled once
-    // PV_{j-1} has.
-    if (j >= 2 && !(ok = pf_wait_warp(sb, sb.pv_done[s], ((j - 2) >> 1) & 1, tmo))) break;
+    // O may be rescaled once PV_{j-1} has completed.
     if (j >= 1 && __any_sync(kFull, resc)) {
       if (!(ok = pf_wait_warp(sb, sb.pv_done[s ^ 1], ((j - 1) >> 1) & 1, tmo))) break;
       tc_fence_after_sync();
@@ -285,38 +289,28 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
     }
 
     const float neg = -m_used;
-    const uint32_t pb = smem + kPfSmemP + s * kPfTileBytes + r * 128;
-    const uint32_t lb = smem + kPfSmemQ + r * 128;
-    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+    float ts[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c8 = 0; c8 < 16; ++c8) {
-      float p[8];
+    for (int c = 0; c < 2; ++c) {
+      uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int c = c8 * 8 + e;
-        const bool valid = !diag || c <= r;
-        p[e] = valid ? ex2_approx(fmaf(__uint_as_float(v[c >> 5][c & 31]), sl2, neg)) : 0.f;
-        ls[e & 3] += p[e];
+      for (int e = 0; e < 16; ++e) {
+        const int k0 = c * 32 + 2 * e;
+        const float p0 = k0 <= lim ? ex2_approx(fmaf(__uint_as_float(v[c][2 * e]), sl2, neg)) : 0.f;
+        const float p1 =
+            k0 + 1 <= lim ? ex2_approx(fmaf(__uint_as_float(v[c][2 * e + 1]), sl2, neg)) : 0.f;
+        ts[(2 * e) & 3] += p0;
+        ts[(2 * e + 1) & 3] += p1;
+        hi[e] = pack_bf16x2(p0, p1);
+        lo[e] = pack_bf16x2(p0 - bf16lo_to_f32(hi[e]), p1 - bf16hi_to_f32(hi[e]));
       }
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(p[2 * e], p[2 * e + 1]);
-      const uint32_t off = (c8 >> 3) * kPfHalfBytes + ((uint32_t)((c8 & 7) ^ (r & 7)) << 4);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pb + off), "r"(w[0]),
-                   "r"(w[1]), "r"(w[2]), "r"(w[3])
-                   : "memory");
-      if (hilo) {
-        uint32_t z[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          z[e] = pack_bf16x2(p[2 * e] - bf16lo_to_f32(w[e]), p[2 * e + 1] - bf16hi_to_f32(w[e]));
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(lb + off), "r"(z[0]),
-                     "r"(z[1]), "r"(z[2]), "r"(z[3])
-                     : "memory");
-      }
+      tmem_st16(sbuf + c * 32, hi);
+      tmem_st16(sbuf + c * 32 + 16, lo);
     }
-    l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-    fence_proxy_async_smem();   // generic-proxy P writes -> tensor-core reads
+    const float T = (ts[0] + ts[1]) + (ts[2] + ts[3]);
+    if (T > kPfLoShare * (l + T)) sb.lo_tile[s] = j + 1;
+    l += T;
+    tmem_wait_st();
     tc_fence_before_sync();
     mbar_arrive(bar_addr(sb.p_full[s]));
   }
@@ -345,9 +339,9 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
 }
 
 // Grid (h_q, B, n_qtiles): block (h, b, z) takes q-tile t = n_qtiles-1-z of
-// head h of sequence b, so the longest rows (most KV tiles) start first and
+// head h of sequence b, so the longest rows (most K/V tiles) start first and
 // the heads of one kv group run side by side (their K/V tiles shared in L2).
-__global__ void __launch_bounds__(kPfThreads, 1)
+__global__ void __launch_bounds__(kPfThreads, 2)
     prefill_tc_bf16(const __grid_constant__ CUtensorMap qmap,
                     const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const PrefillArgs a) {
@@ -374,14 +368,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       raise_status(kStatusSeqlenOverMax);
   }
   if (off + S > a.total_rows) S = a.total_rows > off ? a.total_rows - off : 0;
-  if ((long long)t * kPfRows >= S) return;   // the whole CTA: no rows here
+  const long long row0 = (long long)t * kPfRows;   // first query position of the tile
+  if (row0 >= S) return;                             // the whole CTA: no rows here
   allow_dependent_launch();
 
-  const int nt = t + 1;
-  const bool hilo = (t == 0);
-  const long long qrow = off + (long long)t * kPfRows;
-  const int rows_valid = (int)(S - (long long)t * kPfRows < kPfRows ? S - (long long)t * kPfRows
-                                                                     : kPfRows);
+  const long long rows_left = S - row0;
+  const int rows_valid = rows_left < kPfRows ? (int)rows_left : kPfRows;
+  // K/V tiles covering keys [0, row0 + rows_valid): the causal reach of the tile.
+  const int nt = (int)((row0 + rows_valid + kPfKeys - 1) / kPfKeys);
+  const long long qrow = off + row0;
   const uint32_t smem = (smem_u32(pf_dyn) + 1023u) & ~1023u;
 
   if (threadIdx.x == 0) {
@@ -392,9 +387,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(bar_addr(sb.v_full[s]), 1);
       mbar_init(bar_addr(sb.v_empty[s]), 1);
       mbar_init(bar_addr(sb.s_full[s]), 1);
-      mbar_init(bar_addr(sb.s_free[s]), 4 * 32);
       mbar_init(bar_addr(sb.p_full[s]), 4 * 32);
       mbar_init(bar_addr(sb.pv_done[s]), 1);
+      sb.lo_tile[s] = 0;
     }
     mbar_init(bar_addr(sb.drain), 1);
     sb.abort = 0;
@@ -412,12 +407,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = sb.tmem_base;
 
   if (warp < 4) {
-    pf_softmax(sb, smem, tmem, warp, lane, nt, hilo, a, qrow, rows_valid, h, a.timeout_ns);
+    pf_softmax(sb, tmem, warp, lane, t, nt, a, qrow, rows_valid, h, a.timeout_ns);
   } else if (warp == 4) {
     if (lane == 0)
       pf_producer(sb, smem, &qmap, &kmap, &vmap, h, h / a.G, qrow, off, nt, a.timeout_ns);
   } else {
-    if (lane == 0) pf_mma(sb, smem, tmem, nt, hilo, a.timeout_ns);
+    if (lane == 0) pf_mma(sb, smem, tmem, nt, a.timeout_ns);
   }
   __syncwarp();
   tc_fence_before_sync();
