@@ -234,14 +234,71 @@ __device__ __forceinline__ void pf_rescale_o(uint32_t trow, float f) {
   tmem_wait_st();
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row max (or min, for a negative scale) of the 64 logits, keys c > lim
+// excluded when MASKED.
+template <bool MASKED>
+__device__ __forceinline__ float pf_tile_extreme(const float (&x)[kPfKeys], int lim, float sl2) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+  if (sl2 >= 0.f) {
+#pragma unroll
+    for (int c = 0; c < kPfKeys; c += 4) {
+      const float a0 = (!MASKED || c <= lim) ? x[c] : -INFINITY;
+      const float a1 = (!MASKED || c + 1 <= lim) ? x[c + 1] : -INFINITY;
+      const float a2 = (!MASKED || c + 2 <= lim) ? x[c + 2] : -INFINITY;
+      const float a3 = (!MASKED || c + 3 <= lim) ? x[c + 3] : -INFINITY;
+      m0 = fmax3(m0, a0, a1);
+      m1 = fmax3(m1, a2, a3);
+    }
+    return fmaxf(m0, m1);
+  }
+  m0 = INFINITY, m1 = INFINITY;
+#pragma unroll
+  for (int c = 0; c < kPfKeys; c += 4) {
+    const float a0 = (!MASKED || c <= lim) ? x[c] : INFINITY;
+    const float a1 = (!MASKED || c + 1 <= lim) ? x[c + 1] : INFINITY;
+    const float a2 = (!MASKED || c + 2 <= lim) ? x[c + 2] : INFINITY;
+    const float a3 = (!MASKED || c + 3 <= lim) ? x[c + 3] : INFINITY;
+    m0 = fmin3(m0, a0, a1);
+    m1 = fmin3(m1, a2, a3);
+  }
+  return fminf(m0, m1);
+}
+
+// x <- P = 2^(x * sl2 - m) in place (0 for keys c > lim when MASKED);
+// returns the row's tile mass T.
+template <bool MASKED>
+__device__ __forceinline__ float pf_tile_exp(float (&x)[kPfKeys], int lim, float sl2, float neg) {
+  float ts[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < kPfKeys; ++c) {
+    const float p = ex2_approx(fmaf(x[c], sl2, neg));
+    x[c] = (!MASKED || c <= lim) ? p : 0.f;
+    ts[c & 3] += x[c];
+  }
+  return (ts[0] + ts[1]) + (ts[2] + ts[3]);
+}
+
 // Warps 0-3: thread r owns query row r of the tile (TMEM lane r).  Per K/V
-// tile j: read S_j, mask (key c of the tile is valid while
-// c <= r + 128 t - 64 j), update the row's reference max m (base 2, kept
-// unless the tile's max exceeds it by more than 2^8: then O and the
-// denominator are rescaled), write P = 2^(s * scale * log2e - m) into TMEM
-// as bf16 hi and lo parts, accumulate the fp32 denominator, and flag the
-// block for the lo MMA when this tile holds more than a quarter of the row's
-// mass so far.  Finally O / l is stored for the rows that exist.
+// tile j: read S_j, mask (key c of the tile is causal while
+// c <= r + 128 t - 64 j; only the two tiles that straddle the diagonal
+// need it), update the row's reference max m (base 2, kept unless the
+// tile's max exceeds it by more than 2^8: then O and the denominator are
+// rescaled), write P = 2^(s * scale * log2e - m) into TMEM as bf16 hi
+// parts, and -- in warps where some row's tile mass exceeds a quarter of its
+// running mass, which then also flag the block for the lo MMA -- the lo
+// parts p - hi (zeros elsewhere), and accumulate the fp32 denominator.
+// Finally O / l is stored for the rows that exist.
 __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, int lane, int t,
                                            int nt, const PrefillArgs& a, long long out_row0,
                                            int rows_valid, int h, unsigned long long tmo) {
@@ -255,24 +312,20 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, 
     if (!(ok = pf_wait_warp(sb, sb.s_full[s], (j >> 1) & 1, tmo))) break;
     tc_fence_after_sync();
     const uint32_t sbuf = trow + s * kPfKeys;
-    uint32_t v[2][32];
-    tmem_ld32(sbuf, v[0]);
-    tmem_ld32(sbuf + 32, v[1]);
-    tmem_wait_ld();
-
-    const int lim = r + kPfRows * t - kPfKeys * j;   // keys c <= lim are causal
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    float mn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+    float x[kPfKeys];
+    {
+      uint32_t v[2][32];
+      tmem_ld32(sbuf, v[0]);
+      tmem_ld32(sbuf + 32, v[1]);
+      tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < kPfKeys; ++c) {
-      const float x = __uint_as_float(v[c >> 5][c & 31]);
-      const bool valid = c <= lim;
-      mx[c & 3] = fmaxf(mx[c & 3], valid ? x : -INFINITY);
-      if (sl2 < 0.f) mn[c & 3] = fminf(mn[c & 3], valid ? x : INFINITY);
+      for (int c = 0; c < kPfKeys; ++c) x[c] = __uint_as_float(v[c >> 5][c & 31]);
     }
-    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-    const float tmin = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
-    const float mt = sl2 > 0.f ? tmax * sl2 : (sl2 < 0.f ? tmin * sl2 : 0.f);
+    const bool masked = j >= 2 * t;                  // warp-uniform
+    const int lim = r + kPfRows * t - kPfKeys * j;   // keys c <= lim are causal
+    const float ext = masked ? pf_tile_extreme<true>(x, lim, sl2)
+                             : pf_tile_extreme<false>(x, lim, sl2);
+    const float mt = sl2 != 0.f ? ext * sl2 : 0.f;
     const float m_new = fmaxf(m_used, mt);
     const bool resc = m_new > m_used + kPfRescaleLog2;   // always true on the first tile
     float factor = 1.f;
@@ -288,28 +341,29 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, 
       pf_rescale_o(trow, factor);
     }
 
-    const float neg = -m_used;
-    float ts[4] = {0.f, 0.f, 0.f, 0.f};
+    const float T = masked ? pf_tile_exp<true>(x, lim, sl2, -m_used)
+                           : pf_tile_exp<false>(x, lim, sl2, -m_used);
+    const bool need_lo = T > kPfLoShare * (l + T);
+    l += T;
+    const bool warp_lo = __any_sync(kFull, need_lo);
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int k0 = c * 32 + 2 * e;
-        const float p0 = k0 <= lim ? ex2_approx(fmaf(__uint_as_float(v[c][2 * e]), sl2, neg)) : 0.f;
-        const float p1 =
-            k0 + 1 <= lim ? ex2_approx(fmaf(__uint_as_float(v[c][2 * e + 1]), sl2, neg)) : 0.f;
-        ts[(2 * e) & 3] += p0;
-        ts[(2 * e + 1) & 3] += p1;
-        hi[e] = pack_bf16x2(p0, p1);
-        lo[e] = pack_bf16x2(p0 - bf16lo_to_f32(hi[e]), p1 - bf16hi_to_f32(hi[e]));
-      }
+      for (int e = 0; e < 16; ++e) hi[e] = pack_bf16x2(x[c * 32 + 2 * e], x[c * 32 + 2 * e + 1]);
       tmem_st16(sbuf + c * 32, hi);
+      if (warp_lo) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          lo[e] = pack_bf16x2(x[c * 32 + 2 * e] - bf16lo_to_f32(hi[e]),
+                              x[c * 32 + 2 * e + 1] - bf16hi_to_f32(hi[e]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) lo[e] = 0u;
+      }
       tmem_st16(sbuf + c * 32 + 16, lo);
     }
-    const float T = (ts[0] + ts[1]) + (ts[2] + ts[3]);
-    if (T > kPfLoShare * (l + T)) sb.lo_tile[s] = j + 1;
-    l += T;
+    if (need_lo) sb.lo_tile[s] = j + 1;
     tmem_wait_st();
     tc_fence_before_sync();
     mbar_arrive(bar_addr(sb.p_full[s]));
