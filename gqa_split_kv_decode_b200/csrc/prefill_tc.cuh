@@ -53,6 +53,8 @@ constexpr int kPfSmemBytes = kPfSmemV + 2 * kPfKvBytes;   // 96 KiB
 constexpr int kPfDynSmem = kPfSmemBytes + 1024;          // + alignment slack
 constexpr uint32_t kPfTmemCols = 256;
 constexpr uint32_t kPfColO = 128;
+constexpr int kPfStageStride = kPfD * 4 + 16;          // output staging row, padded
+static_assert(kPfRows * kPfStageStride <= kPfSmemBytes, "output staging must fit");
 constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale: keep the max unless it grew by > 2^8
 constexpr float kPfLoShare = 0.25f;     // a tile above this share of a row's mass takes lo parts
 
@@ -178,9 +180,12 @@ __device__ __forceinline__ void pf_issue_pv(uint32_t tmem, int j, uint32_t vb, b
   }
 }
 
-// Warp 5, one thread.  Issue order: S_0, S_1, then per tile j: PV_j (once P_j
-// is in TMEM; with the lo parts when the softmax asked for them), then
-// S_{j+2} into the same S buffer once PV_j has finished reading P_j there.
+// Warp 5, one thread.  S_0 and S_1 first; then, polling without blocking,
+// S_k as soon as PV_{k-2} has finished reading P_{k-2} from the same TMEM
+// buffer (and K_k is in), and PV_j as soon as P_j and V_j are ready (with
+// the lo parts when the softmax asked for them).  S goes first when both
+// are ready: the softmax waits for it.  No progress for the wait limit
+// aborts the CTA.
 __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem, int nt,
                                        unsigned long long tmo) {
   if (pf_wait(sb, sb.q_full, 0, tmo)) {
@@ -194,24 +199,47 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
       umma_commit(bar_addr(sb.s_full[j]));
       umma_commit(bar_addr(sb.k_empty[j]));
     }
-    for (int j = 0; j < nt && ok; ++j) {
-      const int s = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      if (!pf_wait(sb, sb.p_full[s], par, tmo) || !pf_wait(sb, sb.v_full[s], par, tmo)) break;
-      tc_fence_after_sync();
-      const uint32_t vb = smem + kPfSmemV + s * kPfKvBytes;
-      pf_issue_pv(tmem, j, vb, false, j == 0);
-      if (*reinterpret_cast<volatile int*>(&sb.lo_tile[s]) == j + 1)
-        pf_issue_pv(tmem, j, vb, true, false);
-      umma_commit(bar_addr(sb.pv_done[s]));
-      umma_commit(bar_addr(sb.v_empty[s]));
-      if (j + 2 < nt) {
-        if (!pf_wait(sb, sb.pv_done[s], par, tmo) || !pf_wait(sb, sb.k_full[s], par ^ 1, tmo))
-          break;
-        tc_fence_after_sync();
-        pf_issue_qk(smem, tmem, j + 2);
-        umma_commit(bar_addr(sb.s_full[s]));
-        umma_commit(bar_addr(sb.k_empty[s]));
+    int next_s = 2, next_pv = 0;
+    uint64_t t_progress = globaltimer_ns();
+    while (ok && next_pv < nt) {
+      bool progress = false;
+      if (next_s < nt && next_s - 2 < next_pv) {
+        const int k = next_s, s = k & 1;
+        if (mbar_test_wait(bar_addr(sb.pv_done[s]), ((k - 2) >> 1) & 1) &&
+            mbar_test_wait(bar_addr(sb.k_full[s]), (k >> 1) & 1)) {
+          tc_fence_after_sync();
+          pf_issue_qk(smem, tmem, k);
+          umma_commit(bar_addr(sb.s_full[s]));
+          umma_commit(bar_addr(sb.k_empty[s]));
+          ++next_s;
+          progress = true;
+        }
+      }
+      {
+        const int j = next_pv, s = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (mbar_test_wait(bar_addr(sb.p_full[s]), par) &&
+            mbar_test_wait(bar_addr(sb.v_full[s]), par)) {
+          tc_fence_after_sync();
+          const uint32_t vb = smem + kPfSmemV + s * kPfKvBytes;
+          pf_issue_pv(tmem, j, vb, false, j == 0);
+          if (*reinterpret_cast<volatile int*>(&sb.lo_tile[s]) == j + 1)
+            pf_issue_pv(tmem, j, vb, true, false);
+          umma_commit(bar_addr(sb.pv_done[s]));
+          umma_commit(bar_addr(sb.v_empty[s]));
+          ++next_pv;
+          progress = true;
+        }
+      }
+      if (progress) {
+        t_progress = globaltimer_ns();
+      } else if (*reinterpret_cast<volatile int*>(&sb.abort) ||
+                 globaltimer_ns() - t_progress > tmo) {
+        if (!*reinterpret_cast<volatile int*>(&sb.abort)) {
+          *reinterpret_cast<volatile int*>(&sb.abort) = 1;
+          raise_status(kStatusTimeout);
+        }
+        ok = false;
       }
     }
   }
@@ -299,7 +327,8 @@ __device__ __forceinline__ float pf_tile_exp(float (&x)[kPfKeys], int lim, float
 // running mass, which then also flag the block for the lo MMA -- the lo
 // parts p - hi (zeros elsewhere), and accumulate the fp32 denominator.
 // Finally O / l is stored for the rows that exist.
-__device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, int lane, int t,
+__device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t tmem, int warp,
+                                           int lane, int t,
                                            int nt, const PrefillArgs& a, long long out_row0,
                                            int rows_valid, int h, unsigned long long tmo) {
   const int r = warp * 32 + lane;
@@ -370,25 +399,34 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t tmem, int warp, 
   }
   if (!ok) return;
 
-  // Epilogue: O / l for the rows of this tile that exist.
+  // Epilogue: O / l for the rows of this tile that exist.  Once the last PV
+  // is done no MMA or copy touches shared memory any more, so each thread
+  // stages its normalised row there (rows 528 bytes apart: conflict-free)
+  // and sends it to global memory with one 512-byte bulk copy.
   if (!pf_wait_warp(sb, sb.pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, tmo)) return;
   tc_fence_after_sync();
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  float* dst = a.out + ((out_row0 + r) * a.h_q + h) * (long long)kPfD;
+  const uint32_t srow = smem + r * kPfStageStride;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint32_t o[32];
     tmem_ld32(trow + kPfColO + c * 32, o);
     tmem_wait_ld();
-    if (r < rows_valid) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 val = make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                                       __uint_as_float(o[e + 2]) * inv,
-                                       __uint_as_float(o[e + 3]) * inv);
-        *reinterpret_cast<float4*>(dst + c * 32 + e) = val;
-      }
-    }
+    for (int e = 0; e < 32; e += 4)
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(srow + (c * 32 + e) * 4),
+                   "f"(__uint_as_float(o[e]) * inv), "f"(__uint_as_float(o[e + 1]) * inv),
+                   "f"(__uint_as_float(o[e + 2]) * inv), "f"(__uint_as_float(o[e + 3]) * inv)
+                   : "memory");
+  }
+  fence_proxy_async_smem();   // generic-proxy writes -> bulk-copy reads
+  if (r < rows_valid) {
+    float* dst = a.out + ((out_row0 + r) * a.h_q + h) * (long long)kPfD;
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(srow), "r"(kPfD * 4)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 }
 
@@ -461,7 +499,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   const uint32_t tmem = sb.tmem_base;
 
   if (warp < 4) {
-    pf_softmax(sb, tmem, warp, lane, t, nt, a, qrow, rows_valid, h, a.timeout_ns);
+    pf_softmax(sb, smem, tmem, warp, lane, t, nt, a, qrow, rows_valid, h, a.timeout_ns);
   } else if (warp == 4) {
     if (lane == 0)
       pf_producer(sb, smem, &qmap, &kmap, &vmap, h, h / a.G, qrow, off, nt, a.timeout_ns);
