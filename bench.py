@@ -2,6 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
+--config llama70b_prefill2k | prefill_ragged measures the causal prefill
+kernel instead (one step = one gqa_prefill_attn call; metric TFLOP/s of the
+attended (query, key) pairs against the measured bf16 tensor-core peak).
+
 One step = one call of the fused decode (every step of the path: split
 assignment, TMA-fed K/V stream, logits, online softmax, PV, triplets and the
 log-sum-exp merge) over one batch of the workload, inputs resident in HBM.
@@ -42,6 +46,9 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20
 ROTATE_TOTAL = 1 << 30
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_tc_bf16_persist_llama70b.md")
+PREFILL_PROFILE = os.path.join(ROOT, "profiles", "prefill_tc_bf16_llama70b_prefill2k.md")
+PREFILL_METRIC = "GQA causal prefill attention: TFLOP/s of attended (query, key) pairs and % of B200 bf16 peak; µs/call"
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse_args(argv=None):
@@ -49,7 +56,8 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20000)
     p.add_argument("--warmup", type=int, default=50)
-    p.add_argument("--config", default="llama70b", choices=sorted(workloads.CONFIGS))
+    p.add_argument("--config", default="llama70b",
+                   choices=sorted(workloads.CONFIGS) + sorted(workloads.PREFILL_CONFIGS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -92,27 +100,43 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources each profiled kernel is compiled from (a committed ncu summary
+# stays valid while none of them changes).
+DECODE_SOURCES = ("device_common.cuh", "decode_tc.cuh", "decode_persist.cuh", "split_merge.cuh")
+PREFILL_SOURCES = ("device_common.cuh", "tcgen05.cuh", "prefill_tc.cuh")
+
+
+def kernel_source_hash(names=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gqa_split_kv_decode_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config: str):
+def measured_bf16_peak():
+    """(burst, sustained, source) bf16 dense TFLOP/s."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def profiled_traffic(config: str, summary: str = PROFILE_SUMMARY, sources=DECODE_SOURCES):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel sources and this workload (else None)."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(summary).read()
     except OSError:
         return None
     src = re.search(r"kernel_source_hash:\s*(\w+)", text)
     wl = re.search(r"workload:\s*(\w+)", text)
     tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not (src and wl and tr) or src.group(1) != kernel_source_hash() or wl.group(1) != config:
+    if not (src and wl and tr) or src.group(1) != kernel_source_hash(sources) or wl.group(1) != config:
         return None
     return int(tr.group(1))
 
@@ -452,13 +476,249 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------------ prefill arm
+
+def prefill_desc(w) -> str:
+    sl = w.seqlens.tolist()
+    lens = f"S={sl[0]}" if len(set(sl)) == 1 else f"S_b in [{min(sl)}, {max(sl)}] (seeded)"
+    return (f"{w.name}: causal prefill, B={len(sl)}, {lens}, h_q={w.h_q}, h_kv={w.h_kv}, "
+            f"d_head={w.d}, bf16 q/k/v, fp32 out")
+
+
+def prefill_items(w, n: int, start: int):
+    """n (b, h, i) output rows of the workload, spread over all of them."""
+    sl = w.seqlens.tolist()
+    off = np.concatenate([[0], np.cumsum(sl)])
+    total = int(off[-1]) * w.h_q
+    items = []
+    for k in range(n):
+        x = ((start + k) * 7919) % total        # a fixed stride walk over (row, head)
+        row, h = divmod(x, w.h_q)
+        b = int(np.searchsorted(off, row, side="right") - 1)
+        items.append((b, h, int(row - off[b])))
+    return items
+
+
+def prefill_item_flops(w, items) -> float:
+    return float(sum(4 * w.d * (i + 1) for _, _, i in items))
+
+
+def prefill_cpu_baseline(w, budget_s: float):
+    import oracle
+    cores = os.cpu_count() or 1
+    n = max(cores, 64)
+    t0 = time.perf_counter()
+    oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=prefill_items(w, n, 0))
+    per_item = (time.perf_counter() - t0) / n
+    n_run = int(max(n, budget_s / max(per_item, 1e-9)))
+    items = prefill_items(w, n_run, n)
+    t0 = time.perf_counter()
+    oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=items)
+    dt = time.perf_counter() - t0
+    return {"value": round(prefill_item_flops(w, items) / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": cores, "kind": "oracle",
+            "sample": f"{n_run} (sequence, head, position) output rows of the workload (fp64 two-pass, "
+                      f"{dt:.1f} s); FLOPs = 4 d (i + 1) per row",
+            "seconds": round(dt, 2)}
+
+
+def run_prefill(args, rank, world, local_rank):
+    import gqa_split_kv_decode_b200 as gk
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = workloads.generate_prefill(args.config)
+    flops = w.flops
+    one = sum(t.numel() * t.element_size() for t in (w.q, w.k, w.v)) + w.q.numel() * 4
+    n_copies = max(1, math.ceil(ROTATE_TOTAL / one))
+    qs = [w.q.to(device) for _ in range(n_copies)]
+    ks = [w.k.to(device) for _ in range(n_copies)]
+    vs = [w.v.to(device) for _ in range(n_copies)]
+    outs = [torch.empty(w.q.shape, dtype=torch.float32, device=device) for _ in range(n_copies)]
+    sl = w.seqlens.to(device)
+    ms = w.max_seqlen
+
+    def call(i):
+        c = i % n_copies
+        gk.gqa_prefill_attn(qs[c], ks[c], vs[c], sl, w.scale, max_seqlen=ms, out=outs[c])
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize(device)
+    if gk.get_status(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
+        time.sleep(0.6)
+    K = args.steps
+    stream = torch.cuda.current_stream(device)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_begin()
+    t_start.record(stream)
+    for i in range(K):
+        call(i)
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    if gk.get_status(device) != 0:
+        raise RuntimeError("device status set in the timed region")
+    sampler.stop()
+    clocks = sampler.summary() if rank == 0 else None
+    n_iso = min(K, 100)
+    iso = []
+    for i in range(n_iso):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call(i)
+        b.record(stream)
+        iso.append((a, b))
+    torch.cuda.synchronize(device)
+    iso_ms = max_over_ranks(float(np.median([a.elapsed_time(b) for a, b in iso])), world, device)
+    max_total_ms = max_over_ranks(total_ms, world, device)
+    all_flops = sum_over_ranks(float(flops) * K, world, device)
+
+    # end to end: pinned host q/k/v/seqlens in, fp32 result out, every step
+    E = max(1, min(args.e2e_steps, K))
+    hq, hk, hv, hsl = (t.pin_memory() for t in (w.q, w.k, w.v, w.seqlens))
+    hout = torch.empty(w.q.shape, dtype=torch.float32).pin_memory()
+    dq, dk, dv, dsl = (torch.empty_like(t, device=device) for t in (w.q, w.k, w.v, w.seqlens))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        gk.gqa_prefill_attn(dq, dk, dv, dsl, w.scale, max_seqlen=ms, out=outs[0])
+        hout.copy_(outs[0], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, device)
+    e2e_flops = sum_over_ranks(float(flops), world, device)
+    if rank != 0:
+        return None
+
+    burst, sustained, src = measured_bf16_peak()
+    ms_per_step = max_total_ms / K
+    long_region = max_total_ms > 1000.0
+    peak = sustained if long_region else burst
+    value = all_flops / (max_total_ms * 1e-3) / 1e12
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6),
+        "us_per_call": round(ms_per_step * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
+        "config": {
+            "workload": prefill_desc(w),
+            "flops_per_step": flops,
+            "flop_count": "4 * d_head * h_q * sum_b S_b (S_b + 1) / 2: QK^T and PV over the causal pairs only",
+            "global_batch": len(w.seqlens) * world,
+            "seq_len": ms,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"q/k/v/out rotate among {n_copies} copies ({n_copies * one / 2**30:.2f} GiB)",
+            "accumulate": "fp32 (bf16 tensor-core products in TMEM, fp32 softmax)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_source": (f"{src} MEASURED_PEAKS.json bf16_tflops_sustained (timed region > 1 s)"
+                            if long_region else f"{src} MEASURED_PEAKS.json bf16_tflops (burst)"),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "frac_of_burst_peak": round(achieved / burst, 4),
+            "traffic": profiled_traffic(args.config, PREFILL_PROFILE, PREFILL_SOURCES),
+            "algorithmic_flops_per_launch": flops,
+            "kernel": "prefill_tc_bf16",
+            "launches_per_step": 1,
+            "launch_ms": round(ms_per_step, 6),
+            "isolated_launch_ms": round(iso_ms, 6),
+        },
+        "e2e": {
+            "value": round(e2e_flops / (e2e_ms * 1e-3) / 1e12, 4),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl)),
+            "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+            "ms_per_step": round(e2e_ms, 4),
+            "note": "pinned host q/k/v/seqlens copied in and the fp32 output copied back every step",
+        },
+        "gpu_launches": K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(w, budget_s=12.0)
+    return line
+
+
+def run_prefill_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    w = workloads.generate_prefill(args.config)
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=prefill_items(w, cores, 0))
+    per_item = (time.perf_counter() - t0) / cores
+    steps = args.steps + args.warmup
+    n = int(max(1, 120.0 / max(steps, 1) / max(per_item, 1e-9)))
+    for i in range(args.warmup):
+        oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=prefill_items(w, n, i * n))
+    flops = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        items = prefill_items(w, n, (args.warmup + i) * n)
+        oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=items)
+        flops += prefill_item_flops(w, items)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"{n} (sequence, head, position) output rows per step; FLOPs = 4 d (i + 1) per row"
+    return {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / max(1, args.steps), 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same workload as the GPU arm)",
+        "config": {"workload": prefill_desc(w), "flops_per_step": w.flops},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
     if world != args.gpus and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    prefill = args.config in workloads.PREFILL_CONFIGS
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = (run_prefill_reference if prefill else run_reference)(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return 0
@@ -470,7 +730,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_prefill if prefill else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

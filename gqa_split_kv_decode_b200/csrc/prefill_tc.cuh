@@ -201,6 +201,7 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
     }
     int next_s = 2, next_pv = 0;
     uint64_t t_progress = globaltimer_ns();
+    uint32_t idle = 0;
     while (ok && next_pv < nt) {
       bool progress = false;
       if (next_s < nt && next_s - 2 < next_pv) {
@@ -232,9 +233,11 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
         }
       }
       if (progress) {
-        t_progress = globaltimer_ns();
-      } else if (*reinterpret_cast<volatile int*>(&sb.abort) ||
-                 globaltimer_ns() - t_progress > tmo) {
+        idle = 0;
+      } else if ((++idle & 255u) == 0 &&   // the clock is read now and then only
+                 (*reinterpret_cast<volatile int*>(&sb.abort) ||
+                  (idle == 256 ? (t_progress = globaltimer_ns(), false)
+                               : globaltimer_ns() - t_progress > tmo))) {
         if (!*reinterpret_cast<volatile int*>(&sb.abort)) {
           *reinterpret_cast<volatile int*>(&sb.abort) = 1;
           raise_status(kStatusTimeout);
@@ -395,7 +398,8 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
     if (need_lo) sb.lo_tile[s] = j + 1;
     tmem_wait_st();
     tc_fence_before_sync();
-    mbar_arrive(bar_addr(sb.p_full[s]));
+    __syncwarp();   // one arrival per warp: 128 arrivals on one barrier serialise
+    if (lane == 0) mbar_arrive(bar_addr(sb.p_full[s]));
   }
   if (!ok) return;
 
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       mbar_init(bar_addr(sb.v_full[s]), 1);
       mbar_init(bar_addr(sb.v_empty[s]), 1);
       mbar_init(bar_addr(sb.s_full[s]), 1);
-      mbar_init(bar_addr(sb.p_full[s]), 4 * 32);
+      mbar_init(bar_addr(sb.p_full[s]), 4);
       mbar_init(bar_addr(sb.pv_done[s]), 1);
       sb.lo_tile[s] = 0;
     }
