@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
-    "gqa_prefill_attn", "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "gqa_prefill_attn", "mlo_merge_ranked", "mlo_merge_ranked_raw", "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
 
@@ -64,6 +64,8 @@ _partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c
 _partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci,
                         _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
 _merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
+_merge_ranked = _sig("mlo_merge_ranked", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
+                     ctypes.c_longlong, ctypes.c_longlong, _vp)
 _prefill = _sig("gqa_prefill_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf,
                 _ci, _vp)
 _get_status = _sig("gqa_decode_get_status", _ci, _vp)
@@ -293,6 +295,32 @@ def mlo_merge(m, l, o, out=None) -> torch.Tensor:
     with torch.cuda.device(m.device):
         _check(_merge(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
                       _stream(m.device)), "mlo_merge")
+    return out
+
+
+def mlo_merge_ranked(m, l, o, out=None) -> torch.Tensor:
+    """Merge of triplets gathered from R shards: m, l [R, ..., n], o
+    [R, ..., n, d] -> fp32 [..., d]; a row's splits in rank-major order."""
+    for name, t in (("m", m), ("l", l), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    R, n, d = m.shape[0], o.shape[-2], o.shape[-1]
+    lead = tuple(m.shape[1:-1])
+    if (tuple(m.shape) != (R,) + lead + (n,) or tuple(l.shape) != tuple(m.shape)
+            or tuple(o.shape) != (R,) + lead + (n, d)):
+        raise ValueError("shapes: m, l [R, ..., n]; o [R, ..., n, d]")
+    rows = int(math.prod(lead))
+    out = _out(out, lead + (d,), m.device)
+    return mlo_merge_ranked_raw(m, l, o, out, rows, R, n, d, rows * n, rows * n * d)
+
+
+def mlo_merge_ranked_raw(m, l, o, out, rows, n_ranks, n_splits, d, stride_ml, stride_o):
+    """mlo_merge_ranked on raw views: rank r's m / l block starts r * stride_ml
+    elements after ``m`` / ``l``, its o block r * stride_o after ``o`` (the
+    tensors only supply device addresses)."""
+    with torch.cuda.device(out.device):
+        _check(_merge_ranked(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n_ranks,
+                             n_splits, d, stride_ml, stride_o, _stream(out.device)), "mlo_merge_ranked")
     return out
 
 

@@ -714,6 +714,33 @@ int mlo_merge(const float* m, const float* l, const float* o, float* out, int ro
   return launch_pdl(mlo_merge_kernel<8>, grid, dim3(128), 0, st, m, l, o, out, rows, n_splits, d_head);
 }
 
+int mlo_merge_ranked(const float* m, const float* l, const float* o, float* out, int rows,
+                     int n_ranks, int n_splits, int d_head, long long rank_stride_ml,
+                     long long rank_stride_o, void* stream) {
+  if (rows < 0 || n_ranks < 1 || n_splits < 1 || d_head < 1 || d_head > 256)
+    return GQA_ERR_INVALID_ARG;
+  if ((long long)n_ranks * n_splits > (1 << 20)) return GQA_ERR_INVALID_ARG;
+  if (rows == 0) return GQA_OK;
+  // each rank's block must not overlap the next one's
+  if (n_ranks > 1 && (rank_stride_ml < (long long)rows * n_splits ||
+                      rank_stride_o < (long long)rows * n_splits * d_head))
+    return GQA_ERR_INVALID_ARG;
+  if (!m || !l || !o || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned(m, 4) || !aligned(l, 4) || !aligned(o, 4) || !aligned(out, 4))
+    return GQA_ERR_INVALID_ARG;
+  const dim3 grid((rows + 3) / 4);
+  cudaStream_t st = as_stream(stream);
+  const size_t sml = (size_t)rank_stride_ml, so = (size_t)rank_stride_o;
+  if (d_head <= 64)
+    return launch_pdl(mlo_merge_ranked_kernel<2>, grid, dim3(128), 0, st, m, l, o, out, rows,
+                      n_ranks, n_splits, d_head, sml, so);
+  if (d_head <= 128)
+    return launch_pdl(mlo_merge_ranked_kernel<4>, grid, dim3(128), 0, st, m, l, o, out, rows,
+                      n_ranks, n_splits, d_head, sml, so);
+  return launch_pdl(mlo_merge_ranked_kernel<8>, grid, dim3(128), 0, st, m, l, o, out, rows,
+                    n_ranks, n_splits, d_head, sml, so);
+}
+
 int gqa_decode_auto_splits(int B, int h_q, int h_kv, int d_head, int max_seqlen) {
   return auto_splits(B, h_q, h_kv, d_head, max_seqlen);
 }

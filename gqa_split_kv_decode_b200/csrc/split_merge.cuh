@@ -175,15 +175,35 @@ __device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const f
 // of the first 8 splits are requested together with m and l, and each later
 // batch of 8 before any of its rows is used, so a merge of up to 8 splits
 // costs about one memory round trip.
-template <int MAXK>
+// Split j of a row is at element j of its m / l rows and at o + j * d ...
+struct ContiguousSplits {
+  __device__ __forceinline__ size_t ml(int j) const { return (size_t)j; }
+  __device__ __forceinline__ size_t o(int j, int d) const { return (size_t)j * d; }
+};
+// ... or, for triplets gathered from several shards (shard r's block of
+// rows x n_inner splits `stride_ml` elements after shard r-1's for m and l,
+// `stride_o` for o), split j is split j % n_inner of shard j / n_inner.
+struct ShardedSplits {
+  int n_inner;
+  size_t stride_ml, stride_o;
+  __device__ __forceinline__ size_t ml(int j) const {
+    return (size_t)(j / n_inner) * stride_ml + (size_t)(j % n_inner);
+  }
+  __device__ __forceinline__ size_t o(int j, int d) const {
+    return (size_t)(j / n_inner) * stride_o + (size_t)(j % n_inner) * d;
+  }
+};
+
+template <int MAXK, typename SplitIndex = ContiguousSplits>
 __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
-                                               int n, int d, float* out, int lane) {
+                                               int n, int d, float* out, int lane,
+                                               SplitIndex at = SplitIndex()) {
   constexpr int BATCH = 8;
   float ov[BATCH][MAXK];
   auto load_batch = [&](int j0) {  // o rows j0 .. j0 + BATCH - 1 (those < n)
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
-      const float* oj = o + (size_t)(j0 + u) * d;
+      const float* oj = o + at.o(j0 + u < n ? j0 + u : 0, d);
 #pragma unroll
       for (int k = 0; k < MAXK; ++k) {
         const int dd = lane + 32 * k;
@@ -192,10 +212,10 @@ __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, c
     }
   };
   load_batch(0);  // in flight while the maximum is formed
-  float mi = lane < n ? __ldcg(m + lane) : -INFINITY;
-  float li = lane < n ? __ldcg(l + lane) : 0.f;
+  float mi = lane < n ? __ldcg(m + at.ml(lane)) : -INFINITY;
+  float li = lane < n ? __ldcg(l + at.ml(lane)) : 0.f;
   float M = mi;
-  for (int j = 32 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(m + j));
+  for (int j = 32 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(m + at.ml(j)));
   M = warp_max(M);
 
   float acc[MAXK];
@@ -205,8 +225,8 @@ __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, c
   if (M != -INFINITY) {
     for (int base = 0; base < n; base += 32) {
       if (base > 0) {
-        mi = base + lane < n ? __ldcg(m + base + lane) : -INFINITY;
-        li = base + lane < n ? __ldcg(l + base + lane) : 0.f;
+        mi = base + lane < n ? __ldcg(m + at.ml(base + lane)) : -INFINITY;
+        li = base + lane < n ? __ldcg(l + at.ml(base + lane)) : 0.f;
       }
       const float wi = exp2f((mi - M) * kLog2e);  // 0 for an empty split
       const int cnt = min(32, n - base);
@@ -276,6 +296,25 @@ __global__ void __launch_bounds__(128) mlo_merge_kernel(const float* __restrict_
   if (row >= rows) return;
   merge_row_warp<MAXK>(m + (size_t)row * n, l + (size_t)row * n, o + (size_t)row * n * d, n, d,
                        out + (size_t)row * d, threadIdx.x & 31);
+}
+
+// Merge of triplets gathered from n_ranks shards: rank r's m / l block
+// [rows][n_splits] starts r * stride_ml elements in, its o block
+// [rows][n_splits][d] r * stride_o elements in; a row's splits are taken in
+// rank-major order.  One warp per row.
+template <int MAXK>
+__global__ void __launch_bounds__(128) mlo_merge_ranked_kernel(
+    const float* __restrict__ m, const float* __restrict__ l, const float* __restrict__ o,
+    float* __restrict__ out, int rows, int n_ranks, int n_splits, int d, size_t stride_ml,
+    size_t stride_o) {
+  grid_dependency_wait();
+  allow_dependent_launch();
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const ShardedSplits at{n_splits, stride_ml, stride_o};
+  merge_row_warp<MAXK>(m + (size_t)row * n_splits, l + (size_t)row * n_splits,
+                       o + (size_t)row * n_splits * d, n_ranks * n_splits, d, out + (size_t)row * d,
+                       threadIdx.x & 31, at);
 }
 
 }  // namespace gqa

@@ -216,6 +216,25 @@ GQA_API int mlo_merge(const float *m, const float *l, const float *o, float *out
               int rows, int n_splits, int d_head, void *stream);
 
 /*
+ * The same merge for triplets gathered from n_ranks sequence shards -- the
+ * page's multi-rank form (kernbench "_attention_mesh_mlo.py": replicated Q,
+ * KV sharded along the sequence over ranks, each rank's triplet merged into
+ * the others').  Rank r's triplets are m, l fp32 [rows][n_splits] starting
+ * r * rank_stride_ml floats after m (and l), and o fp32
+ * [rows][n_splits][d_head] starting r * rank_stride_o floats after o -- the
+ * layout an all-gather of every rank's gqa_decode_partial output produces
+ * (stride rows * n_splits and rows * n_splits * d_head when m, l and o are
+ * gathered separately; one common stride when each rank's m, l, o are packed
+ * in one buffer).  A row's splits are summed in rank-major order, so the
+ * result equals mlo_merge over the rank-major concatenation.
+ * 1 <= d_head <= 256, n_ranks * n_splits <= 2^20; with n_ranks > 1 the
+ * strides must keep the ranks' blocks apart.
+ */
+GQA_API int mlo_merge_ranked(const float *m, const float *l, const float *o, float *out,
+                             int rows, int n_ranks, int n_splits, int d_head,
+                             long long rank_stride_ml, long long rank_stride_o, void *stream);
+
+/*
  * Split count the library would choose: the largest n_splits whose grid
  * (n_splits x kv heads x head blocks x B CTAs) still fits on the current
  * device in one wave, capped so a split keeps at least 256 keys when

@@ -165,3 +165,16 @@ def test_prefill_argument_checks(lib, kw, expect):
     rc = lib.gqa_prefill_attn(a["q"], a["k"], a["v"], a["sl"], a["out"], a["B"], a["rows"],
                               a["max_seqlen"], a["h_q"], a["h_kv"], a["d"], a["scale"], a["dtype"], None)
     assert rc == expect
+
+
+def test_ranked_merge_argument_checks(lib):
+    ll = ctypes.c_longlong
+    lib.mlo_merge_ranked.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 4 + [ll, ll, ctypes.c_void_p]
+    ok_args = (FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 128, 4 * 3, 4 * 3 * 128, None)
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE, 0, 2, 3, 128, 12, 1536, None) == OK   # no rows
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE, 4, 0, 3, 128, 12, 1536, None) == INVALID
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 257, 12, 1536, None) == INVALID
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 128, 11, 1536, None) == INVALID  # overlap
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 128, 12, 1535, None) == INVALID
+    assert lib.mlo_merge_ranked(0, *ok_args[1:]) == INVALID
+    assert lib.mlo_merge_ranked(FAKE, FAKE, FAKE, FAKE + 2, *ok_args[4:]) == INVALID           # misaligned
