@@ -15,6 +15,11 @@ timed steps the inputs rotate among copies totalling >= 1 GiB so no step
 reads K/V from L2.  Multi-GPU runs are independent replicas (one per rank,
 weak scaling); time is the max over ranks of CUDA-event time.
 
+--sharded (decode workloads) runs the method's multi-rank form: each rank
+holds a contiguous 1/N slice of every sequence's cache, computes its partial
+triplets, one all-gather exchanges them and every rank merges (strong
+scaling: the value is the whole cache's KV bytes per second).
+
 --impl reference times the CPU oracle (fp64, every host core) on a bounded
 sample of the same workload per step; the GPU is not used.
 """
@@ -62,6 +67,9 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--sharded", action="store_true",
+                   help="decode with every sequence's KV cache split over the ranks (partial triplets, "
+                        "one all-gather, merge) instead of independent replicas")
     return p.parse_args(argv)
 
 
@@ -476,6 +484,112 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------- sharded decode arm
+
+def run_sharded(args, rank, world, local_rank):
+    import gqa_split_kv_decode_b200 as gk
+    from gqa_split_kv_decode_b200 import sharded
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    cfg = workloads.CONFIGS[args.config]
+    w = workloads.generate(cfg)
+    k_loc, v_loc, sl_loc = sharded.shard_packed_cache(w.k, w.v, w.seqlens, rank, world)
+    local_bytes = 2 * k_loc.numel() * k_loc.element_size()
+    n_copies = max(1, math.ceil(ROTATE_TOTAL / max(local_bytes, 1)))
+    q = w.q.to(device)
+    sl = sl_loc.to(device)
+    ks = [k_loc.to(device) for _ in range(n_copies)]
+    vs = [v_loc.to(device) for _ in range(n_copies)]
+    n = gk.auto_splits(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, int(sl_loc.max()) if cfg.B else 0, device)
+    out = torch.empty((cfg.B, cfg.h_q, cfg.d), dtype=torch.float32, device=device)
+
+    def call(i):
+        sharded.sharded_decode(q, ks[i % n_copies], vs[i % n_copies], sl, n, cfg.scale, out=out)
+
+    for i in range(args.warmup):
+        call(i)
+    torch.cuda.synchronize(device)
+    if gk.get_status(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
+        time.sleep(0.6)
+    K = args.steps
+    stream = torch.cuda.current_stream(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_begin()
+    t0.record(stream)
+    for i in range(K):
+        call(i)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    if world > 1:
+        dist.barrier()
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    if gk.get_status(device) != 0:
+        raise RuntimeError("device status set in the timed region")
+    sampler.stop()
+    clocks = sampler.summary() if rank == 0 else None
+
+    E = max(1, min(args.e2e_steps, K))
+    hq, hk, hv, hsl = (t.pin_memory() for t in (w.q, k_loc, v_loc, sl_loc))
+    hout = torch.empty_like(out, device="cpu").pin_memory()
+    dk, dv = torch.empty_like(ks[0]), torch.empty_like(vs[0])
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        sl.copy_(hsl, non_blocking=True)
+        sharded.sharded_decode(q, dk, dv, sl, n, cfg.scale, out=out)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / E, world, device)
+    max_local = max_over_ranks(float(local_bytes), world, device)
+    if rank != 0:
+        return None
+    peak, peak_src = measured_hbm_peak()
+    ms = total_ms / K
+    value = w.kv_bytes / (ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 6), "us_per_call": round(ms * 1e3, 3),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
+        "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes,
+                   "global_batch": cfg.B, "seq_len": cfg.S,
+                   "parallelism": f"sequence-sharded KV over {world} ranks, {n} splits per rank",
+                   "l2": f"each rank's K/V shard rotates among {n_copies} copies"},
+        "roofline": {"bound": "hbm", "achieved": round(max_local / (ms * 1e-3) / 1e9, 2), "peak": peak,
+                     "peak_source": peak_src, "unit": "GB/s",
+                     "frac": round(max_local / (ms * 1e-3) / 1e9 / peak, 4), "traffic": None,
+                     "kernel": "decode_tc_bf16 (partial) + mlo_merge_ranked_kernel, NCCL all-gather between",
+                     "note": "achieved = the largest rank's shard bytes / step time (all-gather included)"},
+        "e2e": {"value": round(w.kv_bytes / (e2e_ms * 1e-3) / 1e9, 3), "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl)),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size(), "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+
+
 # ------------------------------------------------------------ prefill arm
 
 def prefill_desc(w) -> str:
@@ -730,7 +844,8 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = (run_prefill if prefill else run_ours)(args, rank, world, local_rank)
+        arm = run_prefill if prefill else (run_sharded if args.sharded else run_ours)
+        line = arm(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
