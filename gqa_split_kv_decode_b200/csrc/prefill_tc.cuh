@@ -22,7 +22,8 @@
 // TMEM (256 columns, fp32, lane = query row): S0 [0,64), S1 [64,128),
 // O [128,256).  P_j replaces S_j in place: keys 32c..32c+31 of the tile
 // (S columns [32c, 32c+32)) become their bf16 hi parts in columns
-// [32c, 32c+16) and lo parts (p - hi, rounded) in [32c+16, 32c+32).
+// [32c, 32c+16) and lo parts (p - hi, rounded) in [32c+16, 32c+32); S_{j+2}
+// is issued right after PV_j, which reads them (one CTA's MMAs run in order).
 //
 // Precision: the P V product normally takes the hi parts only (one bf16 P).
 // A (128-row, 64-key) block also adds the lo parts -- so its P is exact to
@@ -181,8 +182,8 @@ __device__ __forceinline__ void pf_issue_pv(uint32_t tmem, int j, uint32_t vb, b
 }
 
 // Warp 5, one thread.  S_0 and S_1 first; then, polling without blocking,
-// S_k as soon as PV_{k-2} has finished reading P_{k-2} from the same TMEM
-// buffer (and K_k is in), and PV_j as soon as P_j and V_j are ready (with
+// S_k as soon as PV_{k-2}, which reads P_{k-2} from the same TMEM buffer, is
+// issued (and K_k is in), and PV_j as soon as P_j and V_j are ready (with
 // the lo parts when the softmax asked for them).  S goes first when both
 // are ready: the softmax waits for it.  No progress for the wait limit
 // aborts the CTA.
@@ -204,10 +205,12 @@ __device__ __forceinline__ void pf_mma(PfBars& sb, uint32_t smem, uint32_t tmem,
     uint32_t idle = 0;
     while (ok && next_pv < nt) {
       bool progress = false;
+      // S_k overwrites the TMEM columns of P_{k-2}: it goes in once PV_{k-2}
+      // is issued, since the tensor core executes one CTA's MMAs in issue
+      // order (PV_{k-2} has read P before S_k writes).
       if (next_s < nt && next_s - 2 < next_pv) {
         const int k = next_s, s = k & 1;
-        if (mbar_test_wait(bar_addr(sb.pv_done[s]), ((k - 2) >> 1) & 1) &&
-            mbar_test_wait(bar_addr(sb.k_full[s]), (k >> 1) & 1)) {
+        if (mbar_test_wait(bar_addr(sb.k_full[s]), (k >> 1) & 1)) {
           tc_fence_after_sync();
           pf_issue_qk(smem, tmem, k);
           umma_commit(bar_addr(sb.s_full[s]));
