@@ -154,15 +154,13 @@ __device__ __forceinline__ void pf_producer(PfBars& sb, uint32_t smem, const CUt
 // swizzled 128-byte rows, dims 64..127 in each tile's second half.
 __device__ __forceinline__ void pf_issue_qk(uint32_t smem, uint32_t tmem, int j) {
   constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfKeys, false);
-  const uint32_t qa = smem + kPfSmemQ;
-  const uint32_t kb = smem + kPfSmemK + (j & 1) * kPfKvBytes;
+  const SDesc qa = umma_sdesc_sw128_split(smem + kPfSmemQ, 16, 1024);
+  const SDesc kb = umma_sdesc_sw128_split(smem + kPfSmemK + (j & 1) * kPfKvBytes, 16, 1024);
   const uint32_t d = tmem + (j & 1) * kPfKeys;
 #pragma unroll
-  for (int k = 0; k < kPfD / 16; ++k) {
-    const uint32_t sub = (k & 3) * 32;
-    umma_bf16_ss(d, umma_sdesc_sw128(qa + (k >> 2) * kPfQHalf + sub, 16, 1024),
-                 umma_sdesc_sw128(kb + (k >> 2) * kPfKvHalf + sub, 16, 1024), idesc, k > 0);
-  }
+  for (int k = 0; k < kPfD / 16; ++k)
+    umma_bf16_ss_step(d, qa, ((k >> 2) * kPfQHalf + (k & 3) * 32) >> 4, kb,
+                      ((k >> 2) * kPfKvHalf + (k & 3) * 32) >> 4, idesc, k > 0);
 }
 
 // O (+)= P V_j (M = 128 rows, N = 128 dims, K = 64 keys): P from TMEM (the
@@ -173,12 +171,11 @@ __device__ __forceinline__ void pf_issue_pv(uint32_t tmem, int j, uint32_t vb, b
                                             bool overwrite) {
   constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfD, true);
   const uint32_t p = tmem + (j & 1) * kPfKeys + (lo ? 16 : 0);
+  const SDesc v = umma_sdesc_sw128_split(vb, kPfKvHalf, 1024);
 #pragma unroll
-  for (int k = 0; k < kPfKeys / 16; ++k) {
-    umma_bf16_ts(tmem + kPfColO, p + (k >> 1) * 32 + (k & 1) * 8,
-                 umma_sdesc_sw128(vb + k * 2048, kPfKvHalf, 1024), idesc,
-                 (overwrite && k == 0) ? 0u : 1u);
-  }
+  for (int k = 0; k < kPfKeys / 16; ++k)
+    umma_bf16_ts_step(tmem + kPfColO, p + (k >> 1) * 32 + (k & 1) * 8, v, (k * 2048) >> 4, idesc,
+                      (overwrite && k == 0) ? 0u : 1u);
 }
 
 // Warp 5, one thread.  S_0 and S_1 first; then, polling without blocking,

@@ -39,6 +39,19 @@ __device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t saddr, uint32_t lb
   return d;
 }
 
+// The same descriptor as two 32-bit halves: the low half holds the start
+// address (bits 0-13) and the leading byte offset, so stepping through a
+// tile is one 32-bit add of (byte offset >> 4) to `lo` (no carry leaves the
+// 14-bit field for addresses inside the 228 KiB of shared memory).
+struct SDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc umma_sdesc_sw128_split(uint32_t saddr, uint32_t lbo_bytes,
+                                                        uint32_t sbo_bytes) {
+  const uint64_t d = umma_sdesc_sw128(saddr, lbo_bytes, sbo_bytes);
+  return SDesc{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+
 // ------------------------------------------------------------ MMA issue
 
 // D[tmem] (+)= A[smem] * B[smem], issued by one thread.  `accumulate` = 0
@@ -50,6 +63,36 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// umma_bf16_ss with both descriptors given as 32-bit halves, the start
+// addresses advanced by `a_step` / `b_step` (16-byte units): the issuing
+// thread spends two integer adds per MMA instead of rebuilding descriptors.
+__device__ __forceinline__ void umma_bf16_ss_step(uint32_t d_tmem, SDesc a, uint32_t a_step, SDesc b,
+                                                  uint32_t b_step, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}"
+      ::"r"(d_tmem), "r"(a.lo + a_step), "r"(a.hi), "r"(b.lo + b_step), "r"(b.hi), "r"(idesc),
+        "r"(accumulate)
+      : "memory");
+}
+
+// umma_bf16_ts with the B descriptor given as 32-bit halves (see above).
+__device__ __forceinline__ void umma_bf16_ts_step(uint32_t d_tmem, uint32_t a_tmem, SDesc b,
+                                                  uint32_t b_step, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(b.lo + b_step), "r"(b.hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
