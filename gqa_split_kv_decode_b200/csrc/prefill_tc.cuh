@@ -276,34 +276,33 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// Row max (or min, for a negative scale) of the 64 logits, keys c > lim
-// excluded when MASKED.
+// Max (MIN: min) of the 64 logits, keys c > lim excluded when MASKED: eight
+// independent 3-input chains, then a small tree, so the latency is short.
+template <bool MASKED, bool MIN>
+__device__ __forceinline__ float pf_tile_reduce(const float (&x)[kPfKeys], int lim) {
+  constexpr float kFill = MIN ? INFINITY : -INFINITY;
+  float m[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) m[u] = kFill;
+#pragma unroll
+  for (int c = 0; c < kPfKeys; c += 16) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c0 = c + 2 * u, c1 = c0 + 1;
+      const float a0 = (!MASKED || c0 <= lim) ? x[c0] : kFill;
+      const float a1 = (!MASKED || c1 <= lim) ? x[c1] : kFill;
+      m[u] = MIN ? fmin3(m[u], a0, a1) : fmax3(m[u], a0, a1);
+    }
+  }
+  if (MIN)
+    return fminf(fmin3(fmin3(m[0], m[1], m[2]), fmin3(m[3], m[4], m[5]), m[6]), m[7]);
+  return fmaxf(fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), m[6]), m[7]);
+}
+
+// Row max (or min, for a negative scale) of the 64 logits.
 template <bool MASKED>
 __device__ __forceinline__ float pf_tile_extreme(const float (&x)[kPfKeys], int lim, float sl2) {
-  float m0 = -INFINITY, m1 = -INFINITY;
-  if (sl2 >= 0.f) {
-#pragma unroll
-    for (int c = 0; c < kPfKeys; c += 4) {
-      const float a0 = (!MASKED || c <= lim) ? x[c] : -INFINITY;
-      const float a1 = (!MASKED || c + 1 <= lim) ? x[c + 1] : -INFINITY;
-      const float a2 = (!MASKED || c + 2 <= lim) ? x[c + 2] : -INFINITY;
-      const float a3 = (!MASKED || c + 3 <= lim) ? x[c + 3] : -INFINITY;
-      m0 = fmax3(m0, a0, a1);
-      m1 = fmax3(m1, a2, a3);
-    }
-    return fmaxf(m0, m1);
-  }
-  m0 = INFINITY, m1 = INFINITY;
-#pragma unroll
-  for (int c = 0; c < kPfKeys; c += 4) {
-    const float a0 = (!MASKED || c <= lim) ? x[c] : INFINITY;
-    const float a1 = (!MASKED || c + 1 <= lim) ? x[c + 1] : INFINITY;
-    const float a2 = (!MASKED || c + 2 <= lim) ? x[c + 2] : INFINITY;
-    const float a3 = (!MASKED || c + 3 <= lim) ? x[c + 3] : INFINITY;
-    m0 = fmin3(m0, a0, a1);
-    m1 = fmin3(m1, a2, a3);
-  }
-  return fminf(m0, m1);
+  return sl2 >= 0.f ? pf_tile_reduce<MASKED, false>(x, lim) : pf_tile_reduce<MASKED, true>(x, lim);
 }
 
 // x <- P = 2^(x * sl2 - m) in place (0 for keys c > lim when MASKED);
