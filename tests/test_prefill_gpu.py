@@ -156,3 +156,30 @@ def test_prefill_rejects_unsupported(gk):
     w = prefill_case([10], 4, 2, 128, dtype="f32", seed=16)
     with pytest.raises(gk.GQADecodeError):
         gk.gqa_prefill_attn(w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda())
+
+
+def test_prefill_replays_in_a_cuda_graph(gk):
+    """One launch, no host synchronisation and no allocation when max_seqlen
+    and out are given: the call captures into a CUDA graph, and a replay on
+    new inputs equals a direct call bit for bit."""
+    w1 = prefill_case([700, 300], 16, 2, 128, seed=21)
+    w2 = prefill_case([700, 300], 16, 2, 128, seed=22)
+    q, k, v = w1.q.cuda(), w1.k.cuda(), w1.v.cuda()
+    sl = w1.seqlens.cuda()
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        gk.gqa_prefill_attn(q, k, v, sl, w1.scale, max_seqlen=700, out=out)   # warm-up
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gk.gqa_prefill_attn(q, k, v, sl, w1.scale, max_seqlen=700, out=out)
+    q.copy_(w2.q.cuda()); k.copy_(w2.k.cuda()); v.copy_(w2.v.cuda())
+    g.replay()
+    torch.cuda.synchronize()
+    direct = gk.gqa_prefill_attn(w2.q.cuda(), w2.k.cuda(), w2.v.cuda(), sl, w2.scale, max_seqlen=700)
+    torch.cuda.synchronize()
+    assert gk.get_status() == 0
+    assert torch.equal(out, direct)
