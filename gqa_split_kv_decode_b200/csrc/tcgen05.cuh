@@ -54,19 +54,8 @@ __device__ __forceinline__ SDesc umma_sdesc_sw128_split(uint32_t saddr, uint32_t
 
 // ------------------------------------------------------------ MMA issue
 
-// D[tmem] (+)= A[smem] * B[smem], issued by one thread.  `accumulate` = 0
-// overwrites D.
-__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// umma_bf16_ss with both descriptors given as 32-bit halves, the start
+// D[tmem] (+)= A[smem] * B[smem], issued by one thread; `accumulate` = 0
+// overwrites D.  Both descriptors are given as 32-bit halves, their start
 // addresses advanced by `a_step` / `b_step` (16-byte units): the issuing
 // thread spends two integer adds per MMA instead of rebuilding descriptors.
 __device__ __forceinline__ void umma_bf16_ss_step(uint32_t d_tmem, SDesc a, uint32_t a_step, SDesc b,
@@ -83,7 +72,9 @@ __device__ __forceinline__ void umma_bf16_ss_step(uint32_t d_tmem, SDesc a, uint
       : "memory");
 }
 
-// umma_bf16_ts with the B descriptor given as 32-bit halves (see above).
+// D[tmem] (+)= A[tmem] * B[smem] (A read from tensor memory: lane = row,
+// two consecutive bf16 K elements per 32-bit column, 8 columns per K = 16),
+// the B descriptor given as 32-bit halves (see above).
 __device__ __forceinline__ void umma_bf16_ts_step(uint32_t d_tmem, uint32_t a_tmem, SDesc b,
                                                   uint32_t b_step, uint32_t idesc,
                                                   uint32_t accumulate) {
@@ -93,18 +84,6 @@ __device__ __forceinline__ void umma_bf16_ts_step(uint32_t d_tmem, uint32_t a_tm
       "setp.ne.b32 p, %5, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "r"(b.lo + b_step), "r"(b.hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem] (A read from tensor memory: lane = row,
-// two consecutive bf16 K elements per 32-bit column, 8 columns per K = 16).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -159,14 +138,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
-      : "memory");
-}
-
-// Whole warp: thread i writes 8 consecutive 32-bit columns of its TMEM lane.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 
