@@ -54,6 +54,8 @@ CASES = [
     ([513, 256], 64, 8, 4),                    # Llama-70B head shape
     ([1000], 4, 1, 5),                         # one kv head for all
     ([64, 65, 63, 191, 192, 193], 8, 4, 6),    # lengths around the 64-key tile edges
+    ([1] * 5 + [0] * 3 + [2, 3, 40, 17], 4, 4, 7),   # many very short prompts, empty ones between
+    ([129], 1, 1, 8),                          # one head
 ]
 
 
