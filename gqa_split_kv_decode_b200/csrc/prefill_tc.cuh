@@ -305,18 +305,41 @@ __device__ __forceinline__ float pf_tile_extreme(const float (&x)[kPfKeys], int 
   return sl2 >= 0.f ? pf_tile_reduce<MASKED, false>(x, lim) : pf_tile_reduce<MASKED, true>(x, lim);
 }
 
+// Packed two-lane fp32 arithmetic of sm_100 (one instruction for a pair).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // x <- P = 2^(x * sl2 - m) in place (0 for keys c > lim when MASKED);
-// returns the row's tile mass T.
+// returns the row's tile mass T.  Exponent arguments and sums go two keys
+// per instruction.
 template <bool MASKED>
 __device__ __forceinline__ float pf_tile_exp(float (&x)[kPfKeys], int lim, float sl2, float neg) {
-  float ts[4] = {0.f, 0.f, 0.f, 0.f};
+  const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(neg, neg);
+  float2 ts[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < kPfKeys; ++c) {
-    const float p = ex2_approx(fmaf(x[c], sl2, neg));
-    x[c] = (!MASKED || c <= lim) ? p : 0.f;
-    ts[c & 3] += x[c];
+  for (int c = 0; c < kPfKeys; c += 2) {
+    const float2 arg = ffma2(make_float2(x[c], x[c + 1]), s2, n2);
+    x[c] = (!MASKED || c <= lim) ? ex2_approx(arg.x) : 0.f;
+    x[c + 1] = (!MASKED || c + 1 <= lim) ? ex2_approx(arg.y) : 0.f;
+    ts[(c >> 1) & 1] = fadd2(ts[(c >> 1) & 1], make_float2(x[c], x[c + 1]));
   }
-  return (ts[0] + ts[1]) + (ts[2] + ts[3]);
+  return (ts[0].x + ts[0].y) + (ts[1].x + ts[1].y);
 }
 
 // Warps 0-3: thread r owns query row r of the tile (TMEM lane r).  Per K/V
