@@ -187,6 +187,8 @@ EDGE = [
     (1, 8, 1, 128, [5], 64),              # more splits than keys
     (1, 8, 1, 128, [5000], 1),            # one split
     (3, 8, 8, 64, [0, 0, 0], 4),          # every sequence empty
+    (2, 8, 2, 128, [5000, 3], 1024),      # the most splits a call takes
+    (300, 8, 2, 64, [(37 * i) % 61 for i in range(300)], 2),   # many short sequences
 ]
 
 

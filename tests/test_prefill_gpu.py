@@ -127,6 +127,21 @@ def test_prefill_full_size_sampled(gk, name):
     _assert_close(got[rows, heads], ref)
 
 
+def test_prefill_long_prompt_sampled(gk):
+    """A 32k-token prompt (256 query tiles, the longest first in the grid)
+    and a short one beside it: sampled rows against the oracle."""
+    w = prefill_case([32768, 200], 4, 1, 128, seed=23)
+    got = _run(gk, w)
+    assert gk.get_status() == 0
+    sl = w.seqlens.tolist()
+    items = _sample_items(sl, w.h_q, 700, seed=8)
+    ref = oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=items)
+    off = np.concatenate([[0], np.cumsum(sl)])
+    rows = np.array([(off[b] + i) for b, h, i in items])
+    heads = np.array([h for b, h, i in items])
+    _assert_close(got[rows, heads], ref)
+
+
 def test_prefill_reports_sequence_over_max(gk):
     """S_b above max_seqlen: the status word says so; the rows inside the
     grid are still right."""
