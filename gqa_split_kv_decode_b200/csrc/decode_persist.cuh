@@ -215,15 +215,6 @@ __global__ void __launch_bounds__(NW * 32)
   const uint32_t stage0 = smem_u32(stages) + warp * NS * STAGE;
   const uint32_t bar0 = smem_u32(&full_bar[warp * NS]);
 
-  // q of the first unit is requested before any K/V tile, so it is not
-  // queued behind the whole grid's first burst of TMA traffic.
-  uint32_t qf[NT][STEPS][2];
-  int q_b = -1, q_gy = -1;
-  if (blockIdx.x < A) {
-    load_q_frags<D, NT>(qf, a, first.b, first.gy / a.n_hb, first.gy % a.n_hb, lane);
-    q_b = first.b;
-    q_gy = first.gy;
-  }
 
   // ---- issue cursor: the next tile of this warp's sequence (warp-uniform)
   long long ia = blockIdx.x;
@@ -265,6 +256,16 @@ __global__ void __launch_bounds__(NW * 32)
   };
   for (int s = 0; s < NS && more; ++s) issue_next();
   __syncwarp();
+
+  // q of the first unit (an L2 hit) is requested after the first K/V tiles,
+  // whose DRAM latency it then overlaps.
+  uint32_t qf[NT][STEPS][2];
+  int q_b = -1, q_gy = -1;
+  if (blockIdx.x < A) {
+    load_q_frags<D, NT>(qf, a, first.b, first.gy / a.n_hb, first.gy % a.n_hb, lane);
+    q_b = first.b;
+    q_gy = first.gy;
+  }
 
   WarpAcc<D, NT> acc;
   bool failed = false;
@@ -360,7 +361,9 @@ __global__ void __launch_bounds__(NW * 32)
 }
 
 // Merge of every row's non-empty splits (fused path): one warp per row;
-// a row of an empty sequence is 0.
+// a row of an empty sequence is 0.  The row's first triplets are requested
+// together with its sequence length (every slot of the workspace row may be
+// read; only the n active ones are used).
 template <int MAXK>
 __global__ void __launch_bounds__(128) merge_rows_kernel(const DecodeArgs a, int D) {
   grid_dependency_wait();
@@ -368,16 +371,19 @@ __global__ void __launch_bounds__(128) merge_rows_kernel(const DecodeArgs a, int
   const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= (long long)a.B * a.h_q) return;
   const int b = (int)(row / a.h_q);
-  int L;
-  const int n = active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L);
+  const int S = __ldg(a.seqlens + b);
   const int lane = threadIdx.x & 31;
+  const float *m = a.m + row * a.n_slots, *l = a.l + row * a.n_slots, *o = a.o + row * a.n_slots * D;
+  RowMerge<MAXK> r;
+  r.prefetch(m, l, o, a.n_slots, D, lane, ContiguousSplits());
+  int L;
+  const int n = active_splits(a, seq_keys(a, S).total, L);
   float* out = a.out + row * D;
   if (n == 0) {
     for (int d = lane; d < D; d += 32) out[d] = 0.f;
     return;
   }
-  merge_row_warp<MAXK>(a.m + row * a.n_slots, a.l + row * a.n_slots, a.o + row * a.n_slots * D,
-                       n, D, out, lane);
+  r.finish(m, l, o, n, D, out, lane, ContiguousSplits());
 }
 
 }  // namespace gqa

@@ -168,13 +168,6 @@ __device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const f
   }
 }
 
-// Merges n triplets of one row and normalises: the whole warp cooperates,
-// lane j owning elements j, j+32, ... (d <= 32*MAXK).  Splits are combined
-// strictly in index order, so every element's result is deterministic and
-// identical wherever this function runs.  m in natural-log units.  The o rows
-// of the first 8 splits are requested together with m and l, and each later
-// batch of 8 before any of its rows is used, so a merge of up to 8 splits
-// costs about one memory round trip.
 // Split j of a row is at element j of its m / l rows and at o + j * d ...
 struct ContiguousSplits {
   __device__ __forceinline__ size_t ml(int j) const { return (size_t)j; }
@@ -194,13 +187,24 @@ struct ShardedSplits {
   }
 };
 
+// Merges the n triplets of one row and normalises: the whole warp
+// cooperates, lane j owning elements j, j+32, ... (d <= 32*MAXK).  Splits are
+// combined strictly in index order, so every element's result is
+// deterministic and identical wherever this runs.  m in natural-log units.
+//
+// Two halves, so the first loads can leave before n is known: prefetch()
+// requests the o rows of the first 8 of `n_pre` slots together with their m
+// and l (n_pre >= n: slots in [n, n_pre) are read but never used), finish()
+// merges n splits, requesting each later batch of 8 o rows before any of its
+// rows is used.  A merge of up to 8 splits costs about one memory round trip.
 template <int MAXK, typename SplitIndex = ContiguousSplits>
-__device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
-                                               int n, int d, float* out, int lane,
-                                               SplitIndex at = SplitIndex()) {
-  constexpr int BATCH = 8;
+struct RowMerge {
+  static constexpr int BATCH = 8;
   float ov[BATCH][MAXK];
-  auto load_batch = [&](int j0) {  // o rows j0 .. j0 + BATCH - 1 (those < n)
+  float mi, li;
+
+  __device__ __forceinline__ void load_batch(const float* o, int j0, int n, int d, int lane,
+                                             SplitIndex at) {
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
       const float* oj = o + at.o(j0 + u < n ? j0 + u : 0, d);
@@ -210,47 +214,68 @@ __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, c
         ov[u][k] = (j0 + u < n && dd < d) ? __ldcg(oj + dd) : 0.f;
       }
     }
-  };
-  load_batch(0);  // in flight while the maximum is formed
-  float mi = lane < n ? __ldcg(m + at.ml(lane)) : -INFINITY;
-  float li = lane < n ? __ldcg(l + at.ml(lane)) : 0.f;
-  float M = mi;
-  for (int j = 32 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(m + at.ml(j)));
-  M = warp_max(M);
+  }
 
-  float acc[MAXK];
+  __device__ __forceinline__ void prefetch(const float* m, const float* l, const float* o,
+                                           int n_pre, int d, int lane, SplitIndex at) {
+    load_batch(o, 0, n_pre, d, lane, at);
+    mi = lane < n_pre ? __ldcg(m + at.ml(lane)) : -INFINITY;
+    li = lane < n_pre ? __ldcg(l + at.ml(lane)) : 0.f;
+  }
+
+  __device__ __forceinline__ void finish(const float* m, const float* l, const float* o, int n,
+                                         int d, float* out, int lane, SplitIndex at) {
+    if (lane >= n) {
+      mi = -INFINITY;
+      li = 0.f;
+    }
+    float M = mi;
+    for (int j = 32 + lane; j < n; j += 32) M = fmaxf(M, __ldcg(m + at.ml(j)));
+    M = warp_max(M);
+
+    float acc[MAXK];
 #pragma unroll
-  for (int k = 0; k < MAXK; ++k) acc[k] = 0.f;
-  float L = 0.f;
-  if (M != -INFINITY) {
-    for (int base = 0; base < n; base += 32) {
-      if (base > 0) {
-        mi = base + lane < n ? __ldcg(m + at.ml(base + lane)) : -INFINITY;
-        li = base + lane < n ? __ldcg(l + at.ml(base + lane)) : 0.f;
-      }
-      const float wi = exp2f((mi - M) * kLog2e);  // 0 for an empty split
-      const int cnt = min(32, n - base);
-      for (int j0 = 0; j0 < cnt; j0 += BATCH) {
-        if (base + j0 > 0) load_batch(base + j0);
+    for (int k = 0; k < MAXK; ++k) acc[k] = 0.f;
+    float L = 0.f;
+    if (M != -INFINITY) {
+      for (int base = 0; base < n; base += 32) {
+        if (base > 0) {
+          mi = base + lane < n ? __ldcg(m + at.ml(base + lane)) : -INFINITY;
+          li = base + lane < n ? __ldcg(l + at.ml(base + lane)) : 0.f;
+        }
+        const float wi = exp2f((mi - M) * kLog2e);  // 0 for an empty split
+        const int cnt = min(32, n - base);
+        for (int j0 = 0; j0 < cnt; j0 += BATCH) {
+          if (base + j0 > 0) load_batch(o, base + j0, n, d, lane, at);
 #pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-          const int j = j0 + u;
-          const float wj = __shfl_sync(kFull, wi, j & 31);
-          const float lj = __shfl_sync(kFull, li, j & 31);
-          if (j < cnt) {
-            L = fmaf(lj, wj, L);
+          for (int u = 0; u < BATCH; ++u) {
+            const int j = j0 + u;
+            const float wj = __shfl_sync(kFull, wi, j & 31);
+            const float lj = __shfl_sync(kFull, li, j & 31);
+            if (j < cnt) {
+              L = fmaf(lj, wj, L);
 #pragma unroll
-            for (int k = 0; k < MAXK; ++k) acc[k] = fmaf(ov[u][k], wj, acc[k]);
+              for (int k = 0; k < MAXK; ++k) acc[k] = fmaf(ov[u][k], wj, acc[k]);
+            }
           }
         }
       }
     }
-  }
 #pragma unroll
-  for (int k = 0; k < MAXK; ++k) {
-    const int dd = lane + 32 * k;
-    if (dd < d) out[dd] = L > 0.f ? acc[k] / L : 0.f;
+    for (int k = 0; k < MAXK; ++k) {
+      const int dd = lane + 32 * k;
+      if (dd < d) out[dd] = L > 0.f ? acc[k] / L : 0.f;
+    }
   }
+};
+
+template <int MAXK, typename SplitIndex = ContiguousSplits>
+__device__ __forceinline__ void merge_row_warp(const float* m, const float* l, const float* o,
+                                               int n, int d, float* out, int lane,
+                                               SplitIndex at = SplitIndex()) {
+  RowMerge<MAXK, SplitIndex> r;
+  r.prefetch(m, l, o, n, d, lane, at);
+  r.finish(m, l, o, n, d, out, lane, at);
 }
 
 // Fused finish: after this CTA's triplet is stored, take a ticket for the
