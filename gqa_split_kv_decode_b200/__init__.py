@@ -24,12 +24,17 @@ __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
     "gqa_prefill_attn", "mlo_merge_ranked", "mlo_merge_ranked_raw", "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "checked_build", "bounds_report", "selftest_bounds",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqadecode.so")
+# GQA_DECODE_CHECKED=1 loads the checked build (index checks on the kernels'
+# derived global accesses; same entry points and results).
+_LIB_NAME = "libgqadecode_checked.so" if os.environ.get("GQA_DECODE_CHECKED") == "1" else "libgqadecode.so"
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), _LIB_NAME)
 F32, BF16 = 0, 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE_TIMEOUT, ERR_DEVICE_SEQLEN = range(7)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE_TIMEOUT, ERR_DEVICE_SEQLEN,
+ ERR_DEVICE_BOUNDS) = range(8)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -74,6 +79,9 @@ _launches = _sig("gqa_decode_launches_per_call", _ci, _ci, _ci, _ci, _ci, _ci, _
 _set_timeout = _sig("gqa_decode_set_wait_timeout_ns", _ci, _ull)
 _selftest = _sig("gqa_decode_selftest_wait_timeout", _ci, _ull, _vp)
 _release = _sig("gqa_decode_release", _ci)
+_checked_build = _sig("gqa_decode_checked_build", _ci)
+_bounds_report = _sig("gqa_decode_bounds_report", _ull, _vp)
+_selftest_bounds = _sig("gqa_decode_selftest_bounds", _ci, _vp)
 
 
 class GQADecodeError(RuntimeError):
@@ -364,6 +372,32 @@ def selftest_wait_timeout(ns: int, device=None) -> None:
 
 def release() -> None:
     _check(_release(), "gqa_decode_release")
+
+
+def checked_build() -> bool:
+    """True when the loaded library is the checked build (GQA_DECODE_CHECKED=1)."""
+    return _checked_build() == 1
+
+
+def bounds_report(device=None):
+    """The first failed index check since the last report, as (site, index),
+    or None (always None in the normal build).  Synchronises the stream."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        rec = _bounds_report(_stream(device))
+    if rec == 0:
+        return None
+    if rec == (1 << 64) - 1:
+        raise GQADecodeError(ERR_CUDA, "gqa_decode_bounds_report")
+    rec -= 1
+    return rec >> 56, rec & ((1 << 56) - 1)
+
+
+def selftest_bounds(device=None) -> None:
+    """Checked build: one deliberately failing index check (its store skipped)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        _check(_selftest_bounds(_stream(device)), "gqa_decode_selftest_bounds")
 
 
 def gqa_prefill_attn(q, k, v, seqlens, scale=None, max_seqlen=None, out=None):

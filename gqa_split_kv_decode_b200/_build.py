@@ -1,4 +1,6 @@
-"""Builds libgqadecode.so in-tree with nvcc for sm_100a (B200).
+"""Builds libgqadecode.so in-tree with nvcc for sm_100a (B200), and its
+checked twin libgqadecode_checked.so (-DGQA_CHECKED: index checks on the
+kernels' derived global accesses, reported in the status word).
 
     python gqa_split_kv_decode_b200/_build.py [--verbose-ptxas]
 
@@ -15,6 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgqadecode.so")
+LIB_CHECKED = os.path.join(PKG, "libgqadecode_checked.so")
 SOURCES = [os.path.join(CSRC, "gqa_decode.cu")]
 INCLUDE = os.path.join(ROOT, "include")
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
@@ -30,23 +33,30 @@ FLAGS = [
 ]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in DEPS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not (force or stale()):
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose_ptxas else []), "-o", tmp, *SOURCES]
+def build(force: bool = False, verbose_ptxas: bool = False, checked: bool = False) -> str:
+    """Builds one of the two libraries (the normal one unless `checked`)."""
+    lib = LIB_CHECKED if checked else LIB
+    if not (force or stale(lib)):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [NVCC, *FLAGS, *(["-DGQA_CHECKED"] if checked else []),
+           *(["-Xptxas", "-v"] if verbose_ptxas else []), "-o", tmp, *SOURCES]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False, verbose_ptxas: bool = False) -> list:
+    return [build(force, verbose_ptxas), build(force, False, checked=True)]
 
 
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    for path in build_all(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv):
+        print(path)

@@ -309,7 +309,8 @@ __global__ void __launch_bounds__(NW * 32)
       more = false;
       acc.reset();
     }
-    if (cu.has_new && warp == cu.ntiles % NW) {  // the appended token, after the cached keys
+    if (cu.has_new && warp == cu.ntiles % NW &&  // the appended token, after the cached keys
+        in_bounds((long long)cu.b * a.h_kv + g, (long long)a.B * a.h_kv, kSiteAppend)) {
       const size_t nr = ((size_t)cu.b * a.h_kv + g) * D;
       const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + nr;
       const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + nr;
@@ -330,7 +331,10 @@ __global__ void __launch_bounds__(NW * 32)
       if (warp == 0) {
         xslot_merge<D, NT>(acc, xbuf, lane);
         // ---- store the split's triplet (m in natural-log units)
-        if (lane < 4) {
+        const bool row_ok = in_bounds(   // the block's last head row: its highest slot index
+            (long long)(query_row(a, cu.b, g, min(hb * HB + HB - 1, a.G - 1)) * a.n_slots + cu.slot),
+            (long long)a.B * a.h_q * a.n_slots, kSiteTriplet);
+        if (row_ok && lane < 4) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int gi = hb * HB + nt * 8 + 2 * (lane & 3) + (e & 1);
-              if (gi < a.G) {
+              if (row_ok && gi < a.G) {
                 const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
                 a.o[(query_row(a, cu.b, g, gi) * a.n_slots + cu.slot) * D + d] = acc.o[dt][nt][e];
               }

@@ -39,9 +39,11 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
 #pragma unroll
   for (int hh = 0; hh < HB; ++hh) {
     const int gi = hb * HB + hh;
-    const float* src = qp + query_row(a, b, g, gi < a.G ? gi : 0) * D + lane * PER;
+    const bool ok = gi < a.G && in_bounds((long long)query_row(a, b, g, gi), (long long)a.B * a.h_q,
+                                          kSiteQ);
+    const float* src = qp + query_row(a, b, g, ok ? gi : 0) * D + lane * PER;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) qr[hh][e] = gi < a.G ? src[e] : 0.f;
+    for (int e = 0; e < PER; ++e) qr[hh][e] = ok ? src[e] : 0.f;
   }
 
   float m_run[HB], l_run[HB], o_acc[HB][PER];
@@ -89,7 +91,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
     }
   }
 
-  if (sp.has_new && hb == 0 && warp == 0) {  // write the appended token's row
+  if (sp.has_new && hb == 0 && warp == 0 &&  // write the appended token's row
+      in_bounds(sp.off + sp.cached_hi, (long long)a.B * a.cap, kSiteAppend)) {
     const size_t dst = ((size_t)(sp.off + sp.cached_hi) * a.h_kv + g) * D + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) {

@@ -57,7 +57,8 @@ __device__ __forceinline__ void load_q_frags(uint32_t (&qf)[NT][D / 16][2], cons
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int gi = hb * HB + nt * 8 + (lane >> 2);
-    const bool ok = gi < a.G;
+    const bool ok = gi < a.G && in_bounds((long long)query_row(a, b, g, gi), (long long)a.B * a.h_q,
+                                          kSiteQ);
     const size_t base = (query_row(a, b, g, ok ? gi : 0) * D) / 2 + (lane & 3);
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
@@ -259,7 +260,7 @@ __device__ __forceinline__ void store_new_row(const DecodeArgs& a, const __nv_bf
                                               int lane) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
   const size_t base = ((size_t)dst_row * a.h_kv + g) * D;
-  if (lane < 2 * CH) {
+  if (lane < 2 * CH && in_bounds(dst_row, (long long)a.B * a.cap, kSiteAppend)) {
     const bool isv = lane >= CH;
     const int c = isv ? lane - CH : lane;
     const uint4 val = __ldg(reinterpret_cast<const uint4*>(isv ? vn : kn) + c);
@@ -412,7 +413,8 @@ __global__ void __launch_bounds__(NW * 32)
     for (int i = it; i < last; ++i) mbar_wait_bounded(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns);
     acc.reset();
   }
-  if (sp.has_new && warp == ntiles % NW) {  // the appended token, after the cached keys
+  if (sp.has_new && warp == ntiles % NW &&  // the appended token, after the cached keys
+      in_bounds((long long)b * a.h_kv + g, (long long)a.B * a.h_kv, kSiteAppend)) {
     const size_t nr = ((size_t)b * a.h_kv + g) * D;
     const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + nr;
     const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + nr;

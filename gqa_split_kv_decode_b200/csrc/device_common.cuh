@@ -19,12 +19,51 @@ enum : unsigned {
   kStatusTimeout = 1u,        // a bounded wait ran out
   kStatusNegSeqlen = 2u,      // some S_b < 0 (treated as 0)
   kStatusSeqlenOverMax = 4u,  // S_b above max_seqlen (chunked) or above a padded cache's room
+  kStatusBounds = 8u,         // an index check of the checked build failed (access skipped)
 };
 
 // Per-device status word of this library (one per loaded module).
 __device__ unsigned int g_status;
 
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
+
+// ------------------------------------------------------------ index checks
+//
+// The checked build (-DGQA_CHECKED) tests the element index of every global
+// access whose index the kernels derive (triplet slots, output and query
+// rows, tickets, appended cache rows, prefill output rows) against the extent
+// the host arguments give it.  A failed check sets kStatusBounds, keeps the
+// first failure's site and index in g_bounds_first, and the access is
+// skipped, so a wrong index is reported without ever reaching memory.  In the
+// normal build a check is the constant true and compiles away.
+enum BoundsSite : unsigned {
+  kSiteQ = 1,            // query fragment load
+  kSiteTriplet = 2,      // split triplet store (m, l, o)
+  kSiteMergeRow = 3,     // merge: a row's triplets and its output
+  kSiteTicket = 4,       // fused ticket
+  kSiteAppend = 5,       // appended k / v: source and cache row
+  kSitePrefillOut = 6,   // prefill output row
+  kSiteSelftest = 7,     // the self-test's deliberate failure
+};
+
+#ifdef GQA_CHECKED
+// (site << 56) | (index & 0x00ff'ffff'ffff'ffff) of the first failed check, + 1
+__device__ unsigned long long g_bounds_first;
+
+__device__ __noinline__ bool bounds_fail(unsigned site, long long i) {
+  raise_status(kStatusBounds);
+  const unsigned long long rec =
+      (((unsigned long long)site << 56) | ((unsigned long long)i & 0x00ffffffffffffffull)) + 1;
+  atomicCAS(&g_bounds_first, 0ull, rec);
+  return false;
+}
+
+__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned site) {
+  return (i >= 0 && i < n) ? true : bounds_fail(site, i);
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long, unsigned) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -519,6 +519,12 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
     raise_status(kStatusTimeout);
 }
 
+// Self-test of the index checks: one check whose index equals its extent.
+// It fails, and the store it guards is skipped.
+__global__ void selftest_bounds_kernel(int* sink) {
+  if (threadIdx.x == 0 && in_bounds(1, 1, kSiteSelftest)) *sink = 1;
+}
+
 // ------------------------------------------------------------ prefill
 
 // 3-D view (d = 128, head, row) of a packed bf16 [rows][heads][128] tensor;
@@ -596,6 +602,7 @@ const char* gqa_decode_error_string(int status) {
     case GQA_ERR_WORKSPACE: return "GQA_ERR_WORKSPACE: workspace too small, misaligned or not allocatable";
     case GQA_ERR_DEVICE_TIMEOUT: return "GQA_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
     case GQA_ERR_DEVICE_SEQLEN: return "GQA_ERR_DEVICE_SEQLEN: a kernel saw S_b < 0 or S_b > max_seqlen";
+    case GQA_ERR_DEVICE_BOUNDS: return "GQA_ERR_DEVICE_BOUNDS: an index check of the checked build failed";
     default: return "unknown gqa_status";
   }
 }
@@ -774,8 +781,45 @@ int gqa_decode_get_status(void* stream) {
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return GQA_ERR_CUDA;
   }
   if (word & kStatusTimeout) return GQA_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusBounds) return GQA_ERR_DEVICE_BOUNDS;
   if (word & (kStatusNegSeqlen | kStatusSeqlenOverMax)) return GQA_ERR_DEVICE_SEQLEN;
   return GQA_OK;
+}
+
+int gqa_decode_checked_build(void) {
+#ifdef GQA_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+unsigned long long gqa_decode_bounds_report(void* stream) {
+#ifdef GQA_CHECKED
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ~0ull;
+  unsigned long long rec = 0;
+  if (cudaMemcpyFromSymbol(&rec, g_bounds_first, sizeof(rec)) != cudaSuccess) return ~0ull;
+  if (rec) {
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(g_bounds_first, &zero, sizeof(zero)) != cudaSuccess) return ~0ull;
+  }
+  return rec;
+#else
+  (void)stream;
+  return 0;
+#endif
+}
+
+int gqa_decode_selftest_bounds(void* stream) {
+#ifdef GQA_CHECKED
+  static int* sink = nullptr;  // one int per process, never freed
+  if (!sink && cudaMalloc(&sink, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+  selftest_bounds_kernel<<<1, 32, 0, as_stream(stream)>>>(sink);
+  return after_launch();
+#else
+  (void)stream;
+  return GQA_ERR_UNSUPPORTED;
+#endif
 }
 
 int gqa_decode_set_wait_timeout_ns(unsigned long long timeout_ns) {

@@ -446,7 +446,7 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
                    : "memory");
   }
   fence_proxy_async_smem();   // generic-proxy writes -> bulk-copy reads
-  if (r < rows_valid) {
+  if (r < rows_valid && in_bounds(out_row0 + r, a.total_rows, kSitePrefillOut)) {
     float* dst = a.out + ((out_row0 + r) * a.h_q + h) * (long long)kPfD;
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
                  "r"(srow), "r"(kPfD * 4)

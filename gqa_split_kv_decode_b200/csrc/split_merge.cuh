@@ -39,6 +39,9 @@ struct DecodeArgs {
 
 enum { kPartial = 0, kFused = 1 };
 
+// Tickets in the workspace's fixed ticket area (256 KiB of int32).
+constexpr long long kTicketCount = 65536;
+
 // Keys of one sequence: `cached` rows are read from the cache; `total` keys
 // are attended, the new token being key number `cached` when appending and
 // the sequence's cache rows have room for it.
@@ -129,6 +132,9 @@ __device__ void emit_empty_triplet(const DecodeArgs& a, int b, int g, int hb, in
     const int gi = hb * HB + hh;
     if (gi >= a.G) continue;
     const size_t row = query_row(a, b, g, gi);
+    if (!in_bounds((long long)(row * a.n_slots + slot), (long long)a.B * a.h_q * a.n_slots,
+                   kSiteTriplet))
+      continue;
     a.o[(row * a.n_slots + slot) * D + dd] = 0.f;
     if (dd == 0) {
       a.m[row * a.n_slots + slot] = -INFINITY;
@@ -160,6 +166,9 @@ __device__ void emit_split_triplet(const float* sm_m, const float* sm_l, const f
       }
     }
     const size_t row = query_row(a, b, g, gi);
+    if (!in_bounds((long long)(row * a.n_slots + slot), (long long)a.B * a.h_q * a.n_slots,
+                   kSiteTriplet))
+      continue;
     a.o[(row * a.n_slots + slot) * D + dd] = ov;
     if (dd == 0) {
       a.m[row * a.n_slots + slot] = (M == -INFINITY) ? -INFINITY : M * kLn2;
@@ -289,10 +298,14 @@ __device__ void fused_finish(const DecodeArgs& a, int b, int g, int hb, int n_ac
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    int* t = a.tickets + (size_t)b * gridDim.y + blockIdx.y;
-    const int prev = atomicAdd(t, 1);
-    const int last = (prev == n_active - 1);
-    if (last) atomicExch(t, 0);
+    const long long ti = (long long)b * gridDim.y + blockIdx.y;
+    int last = 0;
+    if (in_bounds(ti, kTicketCount, kSiteTicket)) {
+      int* t = a.tickets + ti;
+      const int prev = atomicAdd(t, 1);
+      last = (prev == n_active - 1);
+      if (last) atomicExch(t, 0);
+    }
     *sm_flag = last;
   }
   __syncthreads();
@@ -303,6 +316,7 @@ __device__ void fused_finish(const DecodeArgs& a, int b, int g, int hb, int n_ac
     const int gi = hb * HB + hh;
     if (gi >= a.G) break;
     const size_t row = query_row(a, b, g, gi);
+    if (!in_bounds((long long)row, (long long)a.B * a.h_q, kSiteMergeRow)) break;
     merge_row_warp<D / 32>(a.m + row * a.n_slots, a.l + row * a.n_slots,
                            a.o + row * a.n_slots * D, n_active, D, a.out + row * D, lane);
   }

@@ -79,7 +79,8 @@ typedef enum {
     GQA_ERR_CUDA = 3,            /* a CUDA runtime / driver call failed */
     GQA_ERR_WORKSPACE = 4,       /* caller workspace too small or misaligned */
     GQA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded wait in a kernel ran out */
-    GQA_ERR_DEVICE_SEQLEN = 6    /* a kernel saw S_b < 0 or S_b > max_seqlen */
+    GQA_ERR_DEVICE_SEQLEN = 6,   /* a kernel saw S_b < 0 or S_b > max_seqlen */
+    GQA_ERR_DEVICE_BOUNDS = 7    /* checked build: an index check failed (access skipped) */
 } gqa_status;
 
 typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
@@ -257,10 +258,35 @@ GQA_API int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, i
 
 /*
  * Synchronises `stream`, then reads and clears this device's status word.
- * Returns GQA_OK, GQA_ERR_DEVICE_TIMEOUT, GQA_ERR_DEVICE_SEQLEN or
- * GQA_ERR_CUDA.
+ * Returns GQA_OK, GQA_ERR_DEVICE_TIMEOUT, GQA_ERR_DEVICE_BOUNDS,
+ * GQA_ERR_DEVICE_SEQLEN (in that order of precedence) or GQA_ERR_CUDA.
  */
 GQA_API int gqa_decode_get_status(void *stream);
+
+/*
+ * The checked build.  libgqadecode_checked.so is this library compiled with
+ * -DGQA_CHECKED: every global access whose element index the kernels derive
+ * (query rows, split triplet slots, merged rows, tickets, the appended
+ * token's source and cache row, prefill output rows) is first tested against
+ * the extent the call's arguments give it.  A failed test sets
+ * GQA_ERR_DEVICE_BOUNDS in the status word, records the first failure, and
+ * skips the access, so a wrong index never reaches memory.  Same entry
+ * points and results otherwise; the normal build compiles the tests away.
+ *
+ * gqa_decode_checked_build: 1 in the checked build, 0 otherwise.
+ * gqa_decode_bounds_report: synchronises `stream`, returns and clears the
+ *   first failed test since the last report as ((site << 56) | index) + 1,
+ *   0 when none failed (always 0 in the normal build), ~0 on a CUDA error.
+ *   Sites: 1 query row, 2 triplet slot, 3 merged row, 4 ticket, 5 appended
+ *   row, 6 prefill output row, 7 the self-test.
+ * gqa_decode_selftest_bounds: launches one test whose index equals its
+ *   extent (the store it guards is skipped); afterwards the status word reads
+ *   GQA_ERR_DEVICE_BOUNDS and the report names site 7.  GQA_ERR_UNSUPPORTED
+ *   in the normal build.
+ */
+GQA_API int gqa_decode_checked_build(void);
+GQA_API unsigned long long gqa_decode_bounds_report(void *stream);
+GQA_API int gqa_decode_selftest_bounds(void *stream);
 
 /* Upper bound, in nanoseconds, on every wait inside the kernels (default
  * 1e9).  A wait that runs out records GQA_ERR_DEVICE_TIMEOUT and the kernel

@@ -62,9 +62,25 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), f"{n} declared in a header but not exported"
 
 
+def test_checked_build_exports_the_same_entry_points(lib):
+    """libgqadecode_checked.so (index checks on) has every declared entry
+    point; each library reports which build it is, and the normal one has no
+    checks to test or report."""
+    checked = ctypes.CDLL(_builder().build(checked=True))
+    for n in declared_functions():
+        assert hasattr(checked, n), f"{n} missing from the checked build"
+    assert checked.gqa_decode_checked_build() == 1
+    assert lib.gqa_decode_checked_build() == 0
+    lib.gqa_decode_selftest_bounds.argtypes = [ctypes.c_void_p]
+    assert lib.gqa_decode_selftest_bounds(None) == UNSUPPORTED
+    lib.gqa_decode_bounds_report.argtypes = [ctypes.c_void_p]
+    lib.gqa_decode_bounds_report.restype = ctypes.c_ulonglong
+    assert lib.gqa_decode_bounds_report(None) == 0
+
+
 def test_version_and_error_strings(lib):
     assert lib.gqa_decode_version() >= 100
-    for code in range(7):
+    for code in range(8):
         assert lib.gqa_decode_error_string(code).startswith(b"GQA_")
     assert b"unknown" in lib.gqa_decode_error_string(99)
 
