@@ -67,6 +67,9 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--seed", type=int, default=None,
+                   help="seed of the synthetic inputs (default: the workload's own, 1000 + config "
+                        "index for decode, 2000 + index for prefill)")
     p.add_argument("--sharded", action="store_true",
                    help="decode with every sequence's KV cache split over the ranks (partial triplets, "
                         "one all-gather, merge) instead of independent replicas")
@@ -234,7 +237,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     cfg = workloads.CONFIGS[args.config]
-    w = workloads.generate(cfg)
+    w = workloads.generate(cfg, seed=args.seed)
     kv_bytes = w.kv_bytes
     n_copies = max(1, math.ceil(ROTATE_TOTAL / kv_bytes))
     q = w.q.to(device)
@@ -300,7 +303,9 @@ def run_ours(args, rank, world, local_rank):
         call(i)
         iso_e[i].record(stream)
     torch.cuda.synchronize(device)
-    iso_ms = float(np.median([a.elapsed_time(b) for a, b in zip(iso_s, iso_e)]))
+    iso_all = [a.elapsed_time(b) for a, b in zip(iso_s, iso_e)]
+    iso_ms = float(np.median(iso_all))
+    iso_p10, iso_p90 = (max_over_ranks(float(np.percentile(iso_all, q)), world, device) for q in (10, 90))
 
     max_total_ms = max_over_ranks(total_ms, world, device)
     max_iso_ms = max_over_ranks(iso_ms, world, device)
@@ -366,6 +371,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
         "config": {
             "workload": workload_desc(cfg),
+            "seed": cfg.seed if args.seed is None else args.seed,
             "kv_bytes_per_step": kv_bytes,
             "global_batch": cfg.B * world,
             "seq_len": cfg.S,
@@ -391,6 +397,7 @@ def run_ours(args, rank, world, local_rank):
                       "together, so the dominant kernel's own rate is at least this)",
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(max_iso_ms, 6),
+            "isolated_launch_ms_p10_p90": [round(iso_p10, 6), round(iso_p90, 6)],
         },
         "e2e": {
             "value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 3),
@@ -452,7 +459,7 @@ def run_reference(args, rank, world):
         return None
     import oracle
     cfg = workloads.CONFIGS[args.config]
-    w = workloads.generate(cfg)
+    w = workloads.generate(cfg, seed=args.seed)
     c = w.cfg
     total = c.B * c.h_q
     cores = os.cpu_count() or 1
@@ -478,7 +485,8 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(1, args.steps), 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, same workload as the GPU arm)",
-        "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes},
+        "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes,
+                   "seed": cfg.seed if args.seed is None else args.seed},
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -494,7 +502,7 @@ def run_sharded(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     cfg = workloads.CONFIGS[args.config]
-    w = workloads.generate(cfg)
+    w = workloads.generate(cfg, seed=args.seed)
     k_loc, v_loc, sl_loc = sharded.shard_packed_cache(w.k, w.v, w.seqlens, rank, world)
     local_bytes = 2 * k_loc.numel() * k_loc.element_size()
     n_copies = max(1, math.ceil(ROTATE_TOTAL / max(local_bytes, 1)))
@@ -575,6 +583,7 @@ def run_sharded(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
         "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes,
+                   "seed": cfg.seed if args.seed is None else args.seed,
                    "global_batch": cfg.B, "seq_len": cfg.S,
                    "parallelism": f"sequence-sharded KV over {world} ranks, {n} splits per rank",
                    "l2": f"each rank's K/V shard rotates among {n_copies} copies"},
@@ -642,7 +651,7 @@ def run_prefill(args, rank, world, local_rank):
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    w = workloads.generate_prefill(args.config)
+    w = workloads.generate_prefill(args.config, seed=args.seed)
     flops = w.flops
     one = sum(t.numel() * t.element_size() for t in (w.q, w.k, w.v)) + w.q.numel() * 4
     n_copies = max(1, math.ceil(ROTATE_TOTAL / one))
@@ -696,7 +705,9 @@ def run_prefill(args, rank, world, local_rank):
         b.record(stream)
         iso.append((a, b))
     torch.cuda.synchronize(device)
-    iso_ms = max_over_ranks(float(np.median([a.elapsed_time(b) for a, b in iso])), world, device)
+    iso_all = [a.elapsed_time(b) for a, b in iso]
+    iso_ms = max_over_ranks(float(np.median(iso_all)), world, device)
+    iso_p10, iso_p90 = (max_over_ranks(float(np.percentile(iso_all, q)), world, device) for q in (10, 90))
     max_total_ms = max_over_ranks(total_ms, world, device)
     all_flops = sum_over_ranks(float(flops) * K, world, device)
 
@@ -751,6 +762,7 @@ def run_prefill(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
         "config": {
             "workload": prefill_desc(w),
+            "seed": "default (2000 + index)" if args.seed is None else args.seed,
             "flops_per_step": flops,
             "flop_count": "4 * d_head * h_q * sum_b S_b (S_b + 1) / 2: QK^T and PV over the causal pairs only",
             "global_batch": len(w.seqlens) * world,
@@ -774,6 +786,7 @@ def run_prefill(args, rank, world, local_rank):
             "launches_per_step": 1,
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(iso_ms, 6),
+            "isolated_launch_ms_p10_p90": [round(iso_p10, 6), round(iso_p90, 6)],
         },
         "e2e": {
             "value": round(e2e_flops / (e2e_ms * 1e-3) / 1e12, 4),
@@ -795,7 +808,7 @@ def run_prefill_reference(args, rank, world):
     if rank != 0:
         return None
     import oracle
-    w = workloads.generate_prefill(args.config)
+    w = workloads.generate_prefill(args.config, seed=args.seed)
     cores = os.cpu_count() or 1
     t0 = time.perf_counter()
     oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=prefill_items(w, cores, 0))
@@ -819,7 +832,8 @@ def run_prefill_reference(args, rank, world):
         "ms_per_step": round(dt * 1e3 / max(1, args.steps), 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, same workload as the GPU arm)",
-        "config": {"workload": prefill_desc(w), "flops_per_step": w.flops},
+        "config": {"workload": prefill_desc(w), "flops_per_step": w.flops,
+                   "seed": "default (2000 + index)" if args.seed is None else args.seed},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

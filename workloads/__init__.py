@@ -234,11 +234,12 @@ def prefill_case(seqlens, h_q, h_kv, d, dtype="bf16", seed=0, std=1.0, scale=Non
                            (1 / math.sqrt(d)) if scale is None else float(scale))
 
 
-def generate_prefill(name: str) -> PrefillWorkload:
+def generate_prefill(name: str, seed: int | None = None) -> PrefillWorkload:
     """The seeded prefill workload ``name``: lengths (ragged: uniform integers
-    in [S_min, S] drawn first from seed 2000 + index), then q, k, v."""
+    in [S_min, S] drawn first from seed 2000 + index, or ``seed``), then q,
+    k, v."""
     c = PREFILL_CONFIGS[name]
-    seed = 2000 + c["index"]
+    seed = 2000 + c["index"] if seed is None else seed
     if c["S_min"] > 0:
         rng = np.random.Generator(np.random.PCG64(seed))
         sl = rng.integers(c["S_min"], c["S"], size=c["B"], endpoint=True).tolist()
