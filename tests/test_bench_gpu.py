@@ -7,8 +7,10 @@ import subprocess
 import sys
 
 import pytest
+import torch
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
