@@ -519,11 +519,13 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
     raise_status(kStatusTimeout);
 }
 
+#ifdef GQA_CHECKED
 // Self-test of the index checks: one check whose index equals its extent.
 // It fails, and the store it guards is skipped.
 __global__ void selftest_bounds_kernel(int* sink) {
   if (threadIdx.x == 0 && in_bounds(1, 1, kSiteSelftest)) *sink = 1;
 }
+#endif
 
 // ------------------------------------------------------------ prefill
 

@@ -452,7 +452,9 @@ __device__ __forceinline__ void pf_softmax(PfBars& sb, uint32_t smem, uint32_t t
                  "r"(srow), "r"(kPfD * 4)
                  : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    // Only the shared-memory reads need to be over before the CTA goes (the
+    // global writes complete with the grid); the slot frees up sooner.
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
 }
 
