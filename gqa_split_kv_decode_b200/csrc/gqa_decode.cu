@@ -814,9 +814,17 @@ unsigned long long gqa_decode_bounds_report(void* stream) {
 
 int gqa_decode_selftest_bounds(void* stream) {
 #ifdef GQA_CHECKED
-  static int* sink = nullptr;  // one int per process, never freed
-  if (!sink && cudaMalloc(&sink, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
-  selftest_bounds_kernel<<<1, 32, 0, as_stream(stream)>>>(sink);
+  // The guarded store's target: one int per device, never freed (the
+  // failing check skips the store, but the pointer is a real one regardless).
+  static std::mutex mu;
+  static int* sink[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!sink[dev] && cudaMalloc(&sink[dev], sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+  }
+  selftest_bounds_kernel<<<1, 32, 0, as_stream(stream)>>>(sink[dev]);
   return after_launch();
 #else
   (void)stream;
