@@ -411,7 +411,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=12.0)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=30.0)
     return line
 
 
@@ -800,7 +800,7 @@ def run_prefill(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = prefill_cpu_baseline(w, budget_s=12.0)
+        line["cpu_baseline"] = prefill_cpu_baseline(w, budget_s=30.0)
     return line
 
 
