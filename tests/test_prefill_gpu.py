@@ -56,6 +56,9 @@ CASES = [
     ([64, 65, 63, 191, 192, 193], 8, 4, 6),    # lengths around the 64-key tile edges
     ([1] * 5 + [0] * 3 + [2, 3, 40, 17], 4, 4, 7),   # many very short prompts, empty ones between
     ([129], 1, 1, 8),                          # one head
+    ([200, 130], 32, 2, 9),                    # group of 16 query heads per kv head
+    ([257], 32, 1, 10),                        # group of 32: every head reads one kv head
+    ([2047, 1, 2049], 8, 2, 11),               # lengths either side of a 2048 boundary
 ]
 
 
