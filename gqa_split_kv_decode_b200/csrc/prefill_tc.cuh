@@ -27,7 +27,7 @@
 //
 // Precision: the P V product normally takes the hi parts only (one bf16 P).
 // A (128-row, 64-key) block also adds the lo parts -- so its P is exact to
-// ~2^-17 -- whenever some row's tile mass exceeds a quarter of that row's
+// ~2^-17 -- whenever some row's tile mass exceeds a third of that row's
 // running denominator; that covers every short row and every tile that
 // carries a row's dominant keys, where a single bf16 rounding of the
 // weights would show in the output.
@@ -57,7 +57,7 @@ constexpr uint32_t kPfColO = 128;
 constexpr int kPfStageStride = kPfD * 4 + 16;          // output staging row, padded
 static_assert(kPfRows * kPfStageStride <= kPfSmemBytes, "output staging must fit");
 constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale: keep the max unless it grew by > 2^8
-constexpr float kPfLoShare = 0.25f;     // a tile above this share of a row's mass takes lo parts
+constexpr float kPfLoShare = 1.f / 3;  // a tile above this share of a row's mass takes lo parts
 
 struct PrefillArgs {
   const int32_t* seqlens;   // [B] device
@@ -348,7 +348,7 @@ __device__ __forceinline__ float pf_tile_exp(float (&x)[kPfKeys], int lim, float
 // need it), update the row's reference max m (base 2, kept unless the
 // tile's max exceeds it by more than 2^8: then O and the denominator are
 // rescaled), write P = 2^(s * scale * log2e - m) into TMEM as bf16 hi
-// parts, and -- in warps where some row's tile mass exceeds a quarter of its
+// parts, and -- in warps where some row's tile mass exceeds a third of its
 // running mass, which then also flag the block for the lo MMA -- the lo
 // parts p - hi (zeros elsewhere), and accumulate the fp32 denominator.
 // Finally O / l is stored for the rows that exist.

@@ -38,7 +38,7 @@
  * Numerics: fp32 logits and softmax; P enters the P.V product as bf16, and a
  * block of 128 query rows x 64 keys also adds the rounding remainder of P
  * (a second bf16 part, so P is exact to ~2^-17 there) whenever some row of
- * the block holds more than a quarter of its running softmax mass in those
+ * the block holds more than a third of its running softmax mass in those
  * keys -- every row's first keys, and any tile that carries a row's dominant
  * keys; fp32 accumulation and output.  Tested against the fp64 oracle with
  * |e| <= 2e-3 + 1e-2 |ref| on bf16 inputs.
