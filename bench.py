@@ -59,14 +59,16 @@ FALLBACK_BF16_TFLOPS = 1590.0
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20000)
-    p.add_argument("--warmup", type=int, default=50)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--config", default="llama70b",
                    choices=sorted(workloads.CONFIGS) + sorted(workloads.PREFILL_CONFIGS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="decode: time only the headline workload (skip the per_config object)")
     p.add_argument("--seed", type=int, default=None,
                    help="seed of the synthetic inputs (default: the workload's own, 1000 + config "
                         "index for decode, 2000 + index for prefill)")
@@ -195,11 +197,19 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, window=None):
+        """Median SM clock and the throttle reasons seen in the samples taken
+        during `window` (host wall times (t0, t1)), widened by one sampling
+        period on each side so a region shorter than the period still has
+        its neighbouring samples; all samples when none fall in it."""
         if self.proc is None or not self.lines:
             return None
-        window = [l for (t, l) in self.lines if self.t0 is not None and self.t0 - 0.1 <= t <= (self.t1 or t) + 0.1]
-        rows = window or [l for _, l in self.lines]
+        t0, t1 = window if window is not None else (self.t0, self.t1)
+        rows = []
+        if t0 is not None:
+            rows = [l for (t, l) in self.lines if t0 - 0.25 <= t <= (t1 or t) + 0.25]
+        in_window = bool(rows)
+        rows = rows or [l for _, l in self.lines]
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -217,7 +227,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm), "in_window": bool(window)}
+                "samples": len(sm), "in_window": in_window}
 
 
 # ----------------------------------------------------------------- our arm
@@ -231,68 +241,182 @@ def workload_desc(c) -> str:
             f"{c.dtype} q/k/v, fp32 out")
 
 
+def tensor_sha256(t: torch.Tensor) -> str:
+    """First 16 hex digits of the SHA-256 of a CPU tensor's bytes."""
+    return hashlib.sha256(t.contiguous().view(-1).view(torch.uint8).numpy()).hexdigest()[:16]
+
+
+def input_hashes(w) -> dict:
+    return {name: tensor_sha256(getattr(w, name)) for name in ("q", "k", "v", "seqlens")}
+
+
+def rotation_copies(kv_bytes: int) -> int:
+    """K/V copies the timed steps rotate through: >= 1 GiB in total (so no
+    step finds its K/V in the 126 MB L2), at most 4096 (the tiny workload)."""
+    return max(1, min(4096, math.ceil(ROTATE_TOTAL / max(kv_bytes, 1))))
+
+
+def l2_note(n_copies: int, kv_bytes: int) -> str:
+    return (f"K/V rotate among {n_copies} copies ({n_copies * kv_bytes / 2**30:.2f} GiB); "
+            f"each step's K/V ({kv_bytes / 2**20:.2f} MiB) "
+            + ("exceeds" if kv_bytes > L2_BYTES else "is below") + " the 126 MB L2")
+
+
+def decode_config(cfg, w, world: int, seed) -> dict:
+    """The `config` object of a decode line; both arms print the same one."""
+    n_copies = rotation_copies(w.kv_bytes)
+    return {
+        "workload": workload_desc(cfg),
+        "seed": cfg.seed if seed is None else seed,
+        "kv_bytes_per_step": w.kv_bytes,
+        "global_batch": cfg.B * world,
+        "seq_len": cfg.S,
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        "l2": l2_note(n_copies, w.kv_bytes),
+        "sha256_q_k_v_seqlens": input_hashes(w),
+    }
+
+
+class DecodeRig:
+    """One decode workload resident on the device: rotating K/V copies, the
+    workspace, and the fused and partial + merge calls of step i."""
+
+    def __init__(self, gk, cfg, w, device):
+        self.gk, self.cfg, self.w, self.device = gk, cfg, w, device
+        self.kv_bytes = w.kv_bytes
+        self.n_copies = rotation_copies(self.kv_bytes)
+        self.q = w.q.to(device)
+        self.sl = w.seqlens.to(device)
+        k0, v0 = w.k.to(device), w.v.to(device)
+        self.ks, self.vs = [k0], [v0]
+        if self.n_copies > 1:
+            kk = torch.empty((self.n_copies - 1,) + tuple(k0.shape), dtype=k0.dtype, device=device)
+            vv = torch.empty_like(kk)
+            kk.copy_(k0.unsqueeze(0).expand_as(kk))
+            vv.copy_(v0.unsqueeze(0).expand_as(vv))
+            self.ks += list(kk.unbind(0))
+            self.vs += list(vv.unbind(0))
+        self.out = torch.empty((cfg.B, cfg.h_q, cfg.d), dtype=torch.float32, device=device)
+        self.max_seqlen = w.max_seqlen
+        if cfg.chunk_len:
+            self.n_slots = max(1, -(-self.max_seqlen // cfg.chunk_len))
+            ws = gk.chunked_workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.chunk_len, self.max_seqlen)
+        else:
+            self.n_slots = cfg.n_splits
+            ws = gk.workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.n_splits)
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=device)
+        self.launches = gk.launches_per_call(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, self.n_slots,
+                                             gk.BF16 if cfg.dtype == "bf16" else gk.F32, device)
+        shape = (cfg.B, cfg.h_q, self.n_slots)
+        self.m = torch.empty(shape, dtype=torch.float32, device=device)
+        self.l = torch.empty(shape, dtype=torch.float32, device=device)
+        self.o = torch.empty(shape + (cfg.d,), dtype=torch.float32, device=device)
+
+    def fused(self, i):
+        c, j = self.cfg, i % self.n_copies
+        if c.chunk_len:
+            self.gk.gqa_decode_attn_chunked(self.q, self.ks[j], self.vs[j], self.sl, c.chunk_len,
+                                            self.max_seqlen, c.scale, out=self.out, workspace=self.ws)
+        else:
+            self.gk.gqa_decode_attn(self.q, self.ks[j], self.vs[j], self.sl, c.n_splits, c.scale,
+                                    out=self.out, workspace=self.ws)
+
+    def partial_merge(self, i):
+        c, j = self.cfg, i % self.n_copies
+        if c.chunk_len:
+            self.gk.gqa_decode_partial_chunked(self.q, self.ks[j], self.vs[j], self.sl, c.chunk_len,
+                                               self.max_seqlen, c.scale, m=self.m, l=self.l, o=self.o)
+        else:
+            self.gk.gqa_decode_partial(self.q, self.ks[j], self.vs[j], self.sl, c.n_splits, c.scale,
+                                       m=self.m, l=self.l, o=self.o)
+        self.gk.mlo_merge(self.m, self.l, self.o, out=self.out)
+
+    def kernel_name(self) -> str:
+        if self.cfg.dtype != "bf16":
+            return "decode_simt_f32 (fused)"
+        return "decode_tc_bf16_persist + merge_rows_kernel" if self.launches == 2 else "decode_tc_bf16 (fused)"
+
+
+def timed_steps(call, K: int, W: int, device, world: int):
+    """W untimed warm-up steps, then exactly K steps between CUDA events on
+    the launching stream, bracketed by a barrier and a synchronize on both
+    sides.  Returns (device ms of the K steps, host wall window)."""
+    stream = torch.cuda.current_stream(device)
+    for i in range(W):
+        call(i)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.time()
+    s.record(stream)
+    for i in range(K):
+        call(W + i)
+    e.record(stream)
+    torch.cuda.synchronize(device)
+    h1 = time.time()
+    if world > 1:
+        dist.barrier()
+    return s.elapsed_time(e), (h0, h1)
+
+
+def check_status(gk, device, where: str):
+    status = gk.get_status(device)
+    if status != 0:
+        raise RuntimeError(f"device status {status} {where}")
+
+
+def per_config_entry(gk, name, args, device, sampler, peak):
+    """One more decode workload timed like the headline (same steps and
+    warm-up), on one GPU."""
+    cfg = workloads.CONFIGS[name]
+    w = workloads.generate(cfg, seed=args.seed)
+    rig = DecodeRig(gk, cfg, w, device)
+    ms, win = timed_steps(rig.fused, args.steps, args.warmup, device, 1)
+    check_status(gk, device, f"after timing {name}")
+    us = ms * 1e3 / args.steps
+    gbs = rig.kv_bytes / (us * 1e-6) / 1e9
+    entry = {
+        "workload": workload_desc(cfg),
+        "us_per_call": round(us, 3),
+        "value_gbs": round(gbs, 2),
+        "frac_of_hbm_peak": round(gbs / peak, 4),
+        "kv_bytes_per_step": rig.kv_bytes,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "kernel": rig.kernel_name(),
+        "launches_per_step": rig.launches,
+        "l2": l2_note(rig.n_copies, rig.kv_bytes),
+        "sha256_q_k_v_seqlens": input_hashes(w),
+        "clocks": sampler.summary(win),
+    }
+    del rig, w
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args, rank, world, local_rank):
     import gqa_split_kv_decode_b200 as gk
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    cfg = workloads.CONFIGS[args.config]
-    w = workloads.generate(cfg, seed=args.seed)
-    kv_bytes = w.kv_bytes
-    n_copies = max(1, math.ceil(ROTATE_TOTAL / kv_bytes))
-    q = w.q.to(device)
-    sl = w.seqlens.to(device)
-    ks = [w.k.to(device) for _ in range(n_copies)]
-    vs = [w.v.to(device) for _ in range(n_copies)]
-    out = torch.empty((cfg.B, cfg.h_q, cfg.d), dtype=torch.float32, device=device)
-    if cfg.chunk_len:
-        ws = torch.zeros(gk.chunked_workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.chunk_len,
-                                                   w.max_seqlen), dtype=torch.uint8, device=device)
-        call = lambda i: gk.gqa_decode_attn_chunked(q, ks[i % n_copies], vs[i % n_copies], sl,
-                                                    cfg.chunk_len, w.max_seqlen, cfg.scale, out=out,
-                                                    workspace=ws)
-    else:
-        ws = torch.zeros(gk.workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.n_splits),
-                         dtype=torch.uint8, device=device)
-        call = lambda i: gk.gqa_decode_attn(q, ks[i % n_copies], vs[i % n_copies], sl, cfg.n_splits,
-                                            cfg.scale, out=out, workspace=ws)
-    stream = torch.cuda.current_stream(device)
-    n_slots = max(1, -(-w.max_seqlen // cfg.chunk_len)) if cfg.chunk_len else cfg.n_splits
-    launches = gk.launches_per_call(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, n_slots,
-                                    gk.BF16 if cfg.dtype == "bf16" else gk.F32, device)
-
-    for i in range(args.warmup):
-        call(i)
-    torch.cuda.synchronize(device)
-    if gk.get_status(device) != 0:
-        raise RuntimeError("device status set during warm-up")
-
+    # The clock sampler runs from before the first warm-up step, so the timed
+    # steps follow the warm-up directly (no idle gap before the timed region).
     sampler = ClockSampler(device.index if device.index is not None else 0)
     if rank == 0 and not args.no_clocks:
         sampler.start()
-        time.sleep(0.6)  # let the sampler start before the timed region
+    cfg = workloads.CONFIGS[args.config]
+    w = workloads.generate(cfg, seed=args.seed)
+    kv_bytes = w.kv_bytes
+    rig = DecodeRig(gk, cfg, w, device)
+    stream = torch.cuda.current_stream(device)
 
     K = args.steps
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    sampler.mark_begin()
-    t_start.record(stream)
-    for i in range(K):
-        call(i)
-    t_end.record(stream)
-    torch.cuda.synchronize(device)
-    sampler.mark_end()
-    if world > 1:
-        dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    status = gk.get_status(device)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
-    sampler.stop()
-    clocks = sampler.summary() if rank == 0 else None
+    total_ms, win = timed_steps(rig.fused, K, args.warmup, device, world)
+    check_status(gk, device, "after the timed region")
+    clocks = sampler.summary(win) if rank == 0 else None
 
     # one launch at a time (events around each call; no overlap between calls)
     n_iso = min(K, 200)
@@ -300,12 +424,17 @@ def run_ours(args, rank, world, local_rank):
     iso_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_iso)]
     for i in range(n_iso):
         iso_s[i].record(stream)
-        call(i)
+        rig.fused(i)
         iso_e[i].record(stream)
     torch.cuda.synchronize(device)
     iso_all = [a.elapsed_time(b) for a, b in zip(iso_s, iso_e)]
     iso_ms = float(np.median(iso_all))
     iso_p10, iso_p90 = (max_over_ranks(float(np.percentile(iso_all, q)), world, device) for q in (10, 90))
+
+    # the same workload through the two-call form: gqa_decode_partial + mlo_merge
+    pm_ms, _ = timed_steps(rig.partial_merge, K, args.warmup, device, world)
+    check_status(gk, device, "after timing partial + merge")
+    max_pm_ms = max_over_ranks(pm_ms, world, device)
 
     max_total_ms = max_over_ranks(total_ms, world, device)
     max_iso_ms = max_over_ranks(iso_ms, world, device)
@@ -317,8 +446,8 @@ def run_ours(args, rank, world, local_rank):
     hk = w.k.pin_memory()
     hv = w.v.pin_memory()
     hsl = w.seqlens.pin_memory()
-    hout = torch.empty_like(out, device="cpu").pin_memory()
-    dq, dk, dv, dsl = torch.empty_like(q), torch.empty_like(ks[0]), torch.empty_like(vs[0]), torch.empty_like(sl)
+    hout = torch.empty_like(rig.out, device="cpu").pin_memory()
+    dq, dk, dv, dsl = (torch.empty_like(t, device=device) for t in (w.q, w.k, w.v, w.seqlens))
 
     def e2e_step():
         dq.copy_(hq, non_blocking=True)
@@ -326,16 +455,17 @@ def run_ours(args, rank, world, local_rank):
         dv.copy_(hv, non_blocking=True)
         dsl.copy_(hsl, non_blocking=True)
         if cfg.chunk_len:
-            gk.gqa_decode_attn_chunked(dq, dk, dv, dsl, cfg.chunk_len, w.max_seqlen, cfg.scale, out=out,
-                                       workspace=ws)
+            gk.gqa_decode_attn_chunked(dq, dk, dv, dsl, cfg.chunk_len, w.max_seqlen, cfg.scale,
+                                       out=rig.out, workspace=rig.ws)
         else:
-            gk.gqa_decode_attn(dq, dk, dv, dsl, cfg.n_splits, cfg.scale, out=out, workspace=ws)
-        hout.copy_(out, non_blocking=True)
+            gk.gqa_decode_attn(dq, dk, dv, dsl, cfg.n_splits, cfg.scale, out=rig.out, workspace=rig.ws)
+        hout.copy_(rig.out, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     e0.record(stream)
     for _ in range(E):
@@ -346,14 +476,28 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl))
     d2h = hout.numel() * hout.element_size()
     e2e_bytes = sum_over_ranks(float(kv_bytes), world, device)
+    launches = rig.launches
+    kernel = rig.kernel_name()
+    del rig, dq, dk, dv, dsl
+    torch.cuda.empty_cache()
+
+    peak, peak_src = measured_hbm_peak()
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = {}
+        for name in workloads.CONFIGS:
+            if name != cfg.name:
+                per_config[name] = per_config_entry(gk, name, args, device, sampler, peak)
+    sampler.stop()
 
     if rank != 0:
         return None
 
-    peak, peak_src = measured_hbm_peak()
     ms_per_step = max_total_ms / K
     value = all_bytes / (max_total_ms * 1e-3) / 1e9
     achieved = kv_bytes / (ms_per_step * 1e-3) / 1e9
+    traffic = profiled_traffic(cfg.name)
+    pm_us = max_pm_ms * 1e3 / K
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -369,18 +513,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
-        "config": {
-            "workload": workload_desc(cfg),
-            "seed": cfg.seed if args.seed is None else args.seed,
-            "kv_bytes_per_step": kv_bytes,
-            "global_batch": cfg.B * world,
-            "seq_len": cfg.S,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": (f"K/V rotate among {n_copies} copies ({n_copies * kv_bytes / 2**30:.2f} GiB); "
-                   f"each step's K/V ({kv_bytes / 2**20:.0f} MiB) "
-                   + ("exceeds" if kv_bytes > L2_BYTES else "is below") + " the 126 MB L2"),
-            "accumulate": "fp32 (bf16 tensor-core products, fp32 softmax and merge)",
-        },
+        "config": decode_config(cfg, w, world, args.seed),
+        "accumulate": "fp32 (bf16 tensor-core products, fp32 softmax and merge)",
         "roofline": {
             "bound": "hbm",
             "achieved": round(achieved, 2),
@@ -388,16 +522,27 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_src == "measured" else "fallback",
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic(cfg.name),
+            "traffic": traffic,
+            "traffic_source": ("dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture, read from the "
+                               "committed summary profiles/decode_tc_bf16_persist_llama70b.md (taken on the "
+                               "current kernel sources: their hash matches), not measured in this run")
+                              if traffic is not None else "none: no ncu summary of the current kernel sources",
             "algorithmic_bytes_per_launch": kv_bytes,
-            "kernel": ("decode_tc_bf16_persist + merge_rows_kernel" if launches == 2 else "decode_tc_bf16 (fused)")
-                      if cfg.dtype == "bf16" else "decode_simt_f32",
+            "kernel": kernel,
             "launches_per_step": launches,
             "timing": "CUDA events around the K back-to-back steps of the timed region (a step's launches "
                       "together, so the dominant kernel's own rate is at least this)",
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(max_iso_ms, 6),
             "isolated_launch_ms_p10_p90": [round(iso_p10, 6), round(iso_p90, 6)],
+        },
+        "partial_merge": {
+            "what": "the same workload as gqa_decode_partial (triplets to HBM) + mlo_merge, two calls per step",
+            "us_per_call": round(pm_us, 3),
+            "value_gbs": round(kv_bytes / (pm_us * 1e-6) / 1e9, 2),
+            "frac_of_hbm_peak": round(kv_bytes / (pm_us * 1e-6) / 1e9 / peak, 4),
+            "steps": K,
+            "warmup": args.warmup,
         },
         "e2e": {
             "value": round(e2e_bytes / (e2e_ms * 1e-3) / 1e9, 3),
@@ -410,8 +555,11 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": K * launches,
         "clocks": clocks,
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=30.0)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
+        line["cpu_baseline"]["single_core"] = single_core_baselines(args.seed)
     return line
 
 
@@ -454,6 +602,29 @@ def cpu_baseline(w, budget_s: float):
             "seconds": round(dt, 2)}
 
 
+def single_core_baselines(seed, budget_s: float = 2.0) -> dict:
+    """The oracle on ONE host thread for the tiny, Llama-2-7B and Llama-70B
+    workloads: (b, h) rows for about `budget_s` each, KV GB/s scaled by the
+    rows done."""
+    import oracle
+    res = {}
+    for name in ("tiny", "llama7b", "llama70b"):
+        w = workloads.generate(workloads.CONFIGS[name], seed=seed)
+        c = w.cfg
+        total = c.B * c.h_q
+        done, start, dt = 0, 0, 0.0
+        while dt < budget_s and done < 64 * total:
+            t0 = time.perf_counter()
+            oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale,
+                        items=oracle_sample(w, 1, start), nthreads=1)
+            dt += time.perf_counter() - t0
+            start += 1
+            done += 1
+        res[name] = {"value": round(w.kv_bytes * done / total / dt / 1e9, 4), "unit": UNIT, "cores": 1,
+                     "sample": f"{done} of {total} (b, h) rows, {dt:.2f} s"}
+    return res
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -484,9 +655,9 @@ def run_reference(args, rank, world):
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(1, args.steps), 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded, same workload as the GPU arm)",
-        "config": {"workload": workload_desc(cfg), "kv_bytes_per_step": w.kv_bytes,
-                   "seed": cfg.seed if args.seed is None else args.seed},
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v; no dataset or weights involved)",
+        "config": decode_config(cfg, w, world, args.seed),
+        "accumulate": "fp64 (the CPU oracle: two-pass softmax, no splitting)",
         "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -516,15 +687,14 @@ def run_sharded(args, rank, world, local_rank):
     def call(i):
         sharded.sharded_decode(q, ks[i % n_copies], vs[i % n_copies], sl, n, cfg.scale, out=out)
 
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
     for i in range(args.warmup):
         call(i)
     torch.cuda.synchronize(device)
     if gk.get_status(device) != 0:
         raise RuntimeError("device status set during warm-up")
-    sampler = ClockSampler(device.index if device.index is not None else 0)
-    if rank == 0 and not args.no_clocks:
-        sampler.start()
-        time.sleep(0.6)
     K = args.steps
     stream = torch.cuda.current_stream(device)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -666,15 +836,14 @@ def run_prefill(args, rank, world, local_rank):
         c = i % n_copies
         gk.gqa_prefill_attn(qs[c], ks[c], vs[c], sl, w.scale, max_seqlen=ms, out=outs[c])
 
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0 and not args.no_clocks:
+        sampler.start()
     for i in range(args.warmup):
         call(i)
     torch.cuda.synchronize(device)
     if gk.get_status(device) != 0:
         raise RuntimeError("device status set during warm-up")
-    sampler = ClockSampler(device.index if device.index is not None else 0)
-    if rank == 0 and not args.no_clocks:
-        sampler.start()
-        time.sleep(0.6)
     K = args.steps
     stream = torch.cuda.current_stream(device)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -655,8 +655,17 @@ int gqa_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_ca
   void* scratch = nullptr;
   if (int rc = noalloc_scratch(&scratch)) return rc;
   // The array keeps whatever the previous call left; the tickets must start
-  // at zero, so clear this call's part of the ticket area first.
-  if (cudaMemsetAsync(scratch, 0, n_tickets(s) * sizeof(int), as_stream(stream)) != cudaSuccess) {
+  // at zero, so clear this call's part of the ticket area first.  The
+  // persistent plan merges in its second kernel and reads no ticket, so a
+  // call that takes it needs no clearing.
+  bool uses_tickets = true;
+  if (dtype == GQA_BF16) {
+    const int G = h_q / h_kv, hb = tc_heads_per_cta(G);
+    const long long units = (long long)s.n_slots * h_kv * ((G + hb - 1) / hb) * B;
+    uses_tickets = fused_plan(units, d_head) != kPlanPersistent;
+  }
+  if (uses_tickets &&
+      cudaMemsetAsync(scratch, 0, n_tickets(s) * sizeof(int), as_stream(stream)) != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_CUDA;
   }

@@ -138,8 +138,9 @@ GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_ca
  * launches nothing.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
  * call before any stream capture.  Every call clears the tickets it uses
- * (cudaMemsetAsync on the stream) and then runs the fused kernel; nothing is
- * allocated or freed.  All calls on a device share that device's one array,
+ * (one cudaMemsetAsync on the stream) and then runs the fused kernels; a call
+ * that takes the persistent plan (gqa_decode_launches_per_call == 2) reads no
+ * ticket and skips the clearing.  Nothing is allocated or freed.  All calls on a device share that device's one array,
  * which keeps the last call's contents: calls that overlap on the GPU (for
  * instance on two streams) race and corrupt each other's results, so order
  * them on one stream.

@@ -51,6 +51,14 @@ def test_decode_bench_line():
     assert d["roofline"]["algorithmic_bytes_per_launch"] == d["config"]["kv_bytes_per_step"]
     import workloads
     assert d["config"]["seed"] == workloads.CONFIGS["llama70b"].seed
+    pm = d["partial_merge"]
+    assert pm["us_per_call"] > 0 and pm["steps"] == 200
+    # every other workload, timed the same way
+    assert sorted(d["per_config"]) == sorted(n for n in workloads.CONFIGS if n != "llama70b")
+    for name, e in d["per_config"].items():
+        assert e["steps"] == 200 and e["warmup"] == 3 and e["us_per_call"] > 0
+        assert abs(e["value_gbs"] - e["kv_bytes_per_step"] / (e["us_per_call"] * 1e3)) < 0.01 * e["value_gbs"]
+        assert 0 < e["frac_of_hbm_peak"] < 1.3
 
 
 def test_prefill_bench_line():

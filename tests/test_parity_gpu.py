@@ -136,38 +136,20 @@ def test_ragged_reduced(gk):
     assert_triplets(m.cpu().numpy(), l.cpu().numpy(), o.cpu().numpy(), om, ol, oo, "bf16", "ragged chunks")
 
 
-def _sample_items(w, n_per_b=None, rng_seed=0):
-    c = w.cfg
-    rng = np.random.default_rng(rng_seed)
-    items = []
-    if c.B == 1:
-        for g in range(c.h_kv):  # one query head of every group, at varying offsets in the group
-            items.append((0, g * c.group + (g * 3) % c.group))
-        items.append((0, c.h_q - 1))
-    else:
-        sl = w.seqlens.numpy()
-        bs = sorted({int(np.argmax(sl)), int(np.argmin(sl))} | set(rng.choice(c.B, 6, replace=False).tolist()))
-        for b in bs:
-            items.append((b, int(rng.integers(c.h_q))))
-            items.append((b, int(rng.integers(c.h_q))))
-    return items
-
-
 @pytest.mark.parametrize("name", ["longctx", "ragged"])
-def test_full_size_sampled(gk, name):
-    """The two large workloads at full size in the benchmark's launch
-    configuration; the oracle computes a sample of (b, h) rows one by one."""
+def test_full_size_every_row(gk, name):
+    """The two large workloads (about 4.3 and 4.8 GB of K/V) at full size, in
+    the launch configuration the benchmark times; every output element of
+    every (b, h) row against the oracle (a full fp64 pass takes a few seconds
+    on the host's cores)."""
     w = workloads.generate(CONFIGS[name])
     c = w.cfg
     if c.chunk_len:
         got = run_fused(gk, w, chunk_len=c.chunk_len)
     else:
         got = run_fused(gk, w, n_splits=c.n_splits)
-    items = _sample_items(w)
-    ref = oracle_out(w, items=items)
-    got_s = np.stack([got[b, h] for b, h in items])
-    assert_close(got_s, ref, "bf16", name + " sampled")
-    assert np.isfinite(got).all()
+    ref = oracle_out(w).reshape(c.B, c.h_q, c.d)
+    assert_close(got, ref, "bf16", name + " full size")
 
 
 # ---------------------------------------------------------------- edge cases

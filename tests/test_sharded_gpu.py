@@ -91,3 +91,74 @@ def test_ranked_merge_rejects_overlapping_strides(gk):
     out = torch.empty(4, 64, device="cuda")
     with pytest.raises(gk.GQADecodeError):
         gk.mlo_merge_ranked_raw(m, m, o, out, 4, 2, 3, 64, 11, 4 * 3 * 64)   # 11 < 4 * 3
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, case, q_out):
+    """One rank of the sequence-sharded decode: its shard of every sequence,
+    the library's partial triplets, the all-gather, the ranked merge."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import datetime
+
+    import torch.distributed as dist
+
+    import oracle as orc
+    from gqa_split_kv_decode_b200 import sharded
+    import gqa_split_kv_decode_b200 as gkr
+    from workloads import random_case as rc
+
+    B, hq, hkv, d, seqlens, n, dtype = case
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = rc(B, hq, hkv, d, seqlens, dtype=dtype, seed=sum(seqlens) % 991)
+        c = w.cfg
+        k_loc, v_loc, sl_loc = sharded.shard_packed_cache(w.k, w.v, w.seqlens, rank, world)
+        out = sharded.sharded_decode(w.q.cuda(), k_loc.cuda(), v_loc.cuda(), sl_loc.cuda(), n, c.scale)
+        torch.cuda.synchronize()
+        status = gkr.get_status()
+        ref = orc.attn(w.q, w.k, w.v, w.seqlens, hq, hkv, c.scale).reshape(B, hq, d)
+        got = out.double().cpu().numpy()
+        atol, rtol = TOL[dtype]
+        excess = float((np.abs(got - ref) - (atol + rtol * np.abs(ref))).max())
+        q_out.put((rank, status, excess, bool(np.isfinite(got).all())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case", [
+    (2, 64, 8, 128, [3000, 1234], 4, "bf16"),
+    (3, 16, 2, 64, [0, 777, 5], 2, "f32"),
+], ids=["llama70b_heads_bf16", "ragged_f32"])
+def test_sharded_decode_two_ranks(gk, case):
+    """The product function sharded_decode with two real ranks: two processes
+    on cuda:0 joined by the gloo backend, whose all-gather moves the CUDA
+    triplet buffers through the host.  No kernel of one rank waits on the
+    other, so one GPU serves both.  Every rank must end with the full result
+    (the oracle over the unsharded cache)."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q_out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, case, q_out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        if p.is_alive():
+            p.kill()
+        assert p.exitcode == 0
+    res = sorted(q_out.get(timeout=10) for _ in range(2))
+    assert [r[0] for r in res] == [0, 1]
+    for _, status, excess, finite in res:
+        assert status == 0 and finite
+        assert excess <= 0.0, excess

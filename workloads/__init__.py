@@ -12,12 +12,16 @@ Shapes follow the pages: Llama-2 7B is multi-head (32 heads of 128), Llama-2
                                     rows S_0 + ... + S_{b-1} onwards
     seqlens  int32 [B]
 
-Recipe (numpy PCG64 seeded with 1000 + config index; draws in this order):
-    1. seqlens (ragged config only): integers uniform in [128, 32768];
-    2. q, then k, then v: standard normals in fp32, drawn in chunks of 2**24
-       values, times the config's std, rounded once to the storage dtype
-       (bf16 round-to-nearest-even via torch);
-    3. structure:
+Recipe (seed = 1000 + config index):
+    1. seqlens (ragged config only): integers uniform in [128, 32768], from
+       numpy PCG64(seed) -- the "main" generator of the later steps too;
+    2. q, then k, then v: standard normals in fp32, times the config's std,
+       rounded once to the storage dtype (bf16 round-to-nearest-even via
+       torch).  Each tensor is drawn in chunks of 2**24 values; chunk c of
+       tensor t (q = 0, k = 1, v = 2) comes from its own PCG64 seeded with
+       SeedSequence([seed, t, c]), so the chunks are drawn in parallel and the
+       values do not depend on the thread count;
+    3. structure (from the main generator, in this order):
        - "llama70b": per sequence, round(0.001 * S) distinct key positions;
          for each kv head g, the minimum-norm vector delta with
          Q_g delta = (6 / scale) * 1 (Q_g = the group's bf16 queries) is added
@@ -29,6 +33,8 @@ Recipe (numpy PCG64 seeded with 1000 + config index; draws in this order):
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
 import numpy as np
@@ -108,23 +114,36 @@ def _torch_dtype(name: str):
     return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
 
 
-def _normal(rng: np.random.Generator, shape, std: float, dtype) -> torch.Tensor:
-    """Standard normals x std, drawn in fixed chunks, stored in ``dtype``."""
+def _normal(seed: int, tensor_id: int, shape, std: float, dtype) -> torch.Tensor:
+    """Standard normals x std stored in ``dtype``; chunk c of the flat tensor
+    is drawn from PCG64(SeedSequence([seed, tensor_id, c])), chunks in
+    parallel threads (numpy and torch release the GIL while filling)."""
     out = torch.empty(shape, dtype=dtype)
     flat = out.view(-1)
     n = flat.numel()
-    for s in range(0, n, CHUNK):
-        e = min(n, s + CHUNK)
-        x = rng.standard_normal(e - s, dtype=np.float32)
+
+    def fill(c: int) -> None:
+        s, e = c * CHUNK, min(n, (c + 1) * CHUNK)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tensor_id, c])))
+        x = g.standard_normal(e - s, dtype=np.float32)
         if std != 1.0:
             x *= np.float32(std)
         flat[s:e] = torch.from_numpy(x).to(dtype)
+
+    n_chunks = (n + CHUNK - 1) // CHUNK
+    if n_chunks <= 1:
+        for c in range(n_chunks):
+            fill(c)
+    else:
+        with ThreadPoolExecutor(max_workers=min(n_chunks, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(n_chunks)))
     return out
 
 
 def generate(cfg: Config, seed: int | None = None, seqlens=None) -> Workload:
     """Build the seeded inputs of ``cfg`` (see the module docstring)."""
-    rng = np.random.Generator(np.random.PCG64(cfg.seed if seed is None else seed))
+    seed = cfg.seed if seed is None else seed
+    rng = np.random.Generator(np.random.PCG64(seed))
     if seqlens is not None:
         sl = torch.as_tensor(np.asarray(seqlens, dtype=np.int32))
     elif cfg.S_min > 0:
@@ -133,9 +152,9 @@ def generate(cfg: Config, seed: int | None = None, seqlens=None) -> Workload:
         sl = torch.full((cfg.B,), cfg.S, dtype=torch.int32)
     dt = _torch_dtype(cfg.dtype)
     rows = int(sl.sum())
-    q = _normal(rng, (cfg.B, cfg.h_q, cfg.d), cfg.std, dt)
-    k = _normal(rng, (rows, cfg.h_kv, cfg.d), cfg.std, dt)
-    v = _normal(rng, (rows, cfg.h_kv, cfg.d), cfg.std, dt)
+    q = _normal(seed, 0, (cfg.B, cfg.h_q, cfg.d), cfg.std, dt)
+    k = _normal(seed, 1, (rows, cfg.h_kv, cfg.d), cfg.std, dt)
+    v = _normal(seed, 2, (rows, cfg.h_kv, cfg.d), cfg.std, dt)
 
     if cfg.bias_frac > 0.0:
         off = 0
@@ -221,15 +240,15 @@ PREFILL_CONFIGS = {
 
 def prefill_case(seqlens, h_q, h_kv, d, dtype="bf16", seed=0, std=1.0, scale=None,
                  name="case") -> PrefillWorkload:
-    """N(0, std^2) causal-prefill inputs with explicit lengths.  Draws q, then
-    k, then v (PCG64 ``seed``, fp32 chunks, rounded once to ``dtype``)."""
-    rng = np.random.Generator(np.random.PCG64(seed))
+    """N(0, std^2) causal-prefill inputs with explicit lengths: q, k, v drawn
+    like the decode tensors (fp32 chunks from PCG64(SeedSequence([seed,
+    tensor, chunk])), rounded once to ``dtype``)."""
     sl = torch.as_tensor(np.asarray(list(seqlens), dtype=np.int32))
     rows = int(sl.sum())
     dt = _torch_dtype(dtype)
-    q = _normal(rng, (rows, h_q, d), std, dt)
-    k = _normal(rng, (rows, h_kv, d), std, dt)
-    v = _normal(rng, (rows, h_kv, d), std, dt)
+    q = _normal(seed, 0, (rows, h_q, d), std, dt)
+    k = _normal(seed, 1, (rows, h_kv, d), std, dt)
+    v = _normal(seed, 2, (rows, h_kv, d), std, dt)
     return PrefillWorkload(name, q, k, v, sl, h_q, h_kv, d,
                            (1 / math.sqrt(d)) if scale is None else float(scale))
 
