@@ -67,6 +67,10 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--seq-len", type=int, default=None,
+                   help="decode: override the workload's S (the ragged workload's upper bound), "
+                        "e.g. a smaller case of the same structure for an ncu capture")
+    p.add_argument("--batch", type=int, default=None, help="decode: override the workload's B")
     p.add_argument("--no-per-config", action="store_true",
                    help="decode: time only the headline workload (skip the per_config object)")
     p.add_argument("--seed", type=int, default=None,
@@ -231,6 +235,17 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- our arm
+
+def decode_cfg(args):
+    """The decode workload of --config, with --seq-len / --batch applied."""
+    cfg = workloads.CONFIGS[args.config]
+    over = {}
+    if args.seq_len is not None:
+        over["S"] = args.seq_len
+    if args.batch is not None:
+        over["B"] = args.batch
+    return workloads.scaled(cfg.name, **over) if over else cfg
+
 
 def workload_desc(c) -> str:
     if c.chunk_len:
@@ -407,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(device.index if device.index is not None else 0)
     if rank == 0 and not args.no_clocks:
         sampler.start()
-    cfg = workloads.CONFIGS[args.config]
+    cfg = decode_cfg(args)
     w = workloads.generate(cfg, seed=args.seed)
     kv_bytes = w.kv_bytes
     rig = DecodeRig(gk, cfg, w, device)
@@ -483,7 +498,7 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_src = measured_hbm_peak()
     per_config = None
-    if world == 1 and not args.no_per_config:
+    if world == 1 and not args.no_per_config and cfg == workloads.CONFIGS.get(cfg.name):
         per_config = {}
         for name in workloads.CONFIGS:
             if name != cfg.name:
@@ -496,7 +511,7 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = max_total_ms / K
     value = all_bytes / (max_total_ms * 1e-3) / 1e9
     achieved = kv_bytes / (ms_per_step * 1e-3) / 1e9
-    traffic = profiled_traffic(cfg.name)
+    traffic = profiled_traffic(cfg.name) if cfg == workloads.CONFIGS.get(cfg.name) else None
     pm_us = max_pm_ms * 1e3 / K
     line = {
         "metric": METRIC,
@@ -629,7 +644,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     import oracle
-    cfg = workloads.CONFIGS[args.config]
+    cfg = decode_cfg(args)
     w = workloads.generate(cfg, seed=args.seed)
     c = w.cfg
     total = c.B * c.h_q
@@ -672,7 +687,7 @@ def run_sharded(args, rank, world, local_rank):
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    cfg = workloads.CONFIGS[args.config]
+    cfg = decode_cfg(args)
     w = workloads.generate(cfg, seed=args.seed)
     k_loc, v_loc, sl_loc = sharded.shard_packed_cache(w.k, w.v, w.seqlens, rank, world)
     local_bytes = 2 * k_loc.numel() * k_loc.element_size()

@@ -107,28 +107,59 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"q/k/v must be bf16 or fp32, got {t.dtype}")
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device) -> int:
-    return torch.cuda.current_stream(device).cuda_stream
+    """cudaStream_t of torch's current stream on ``device`` (a torch.device
+    or an index)."""
+    idx = device if isinstance(device, int) else device.index
+    if idx is None:
+        idx = torch.cuda.current_device()
+    if _raw_stream is not None:
+        return _raw_stream(idx)
+    return torch.cuda.current_stream(idx).cuda_stream
+
+
+def _on(idx: int, fn, *args) -> int:
+    """Calls the C entry point with device ``idx`` current (switching only
+    when another device is)."""
+    if torch.cuda.current_device() == idx:
+        return fn(*args)
+    with torch.cuda.device(idx):
+        return fn(*args)
+
+
+_NAMES = ("q", "k_cache", "v_cache", "seqlens")
 
 
 def _inputs(q, k_cache, v_cache, seqlens):
-    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("seqlens", seqlens)):
+    """Checks the decode inputs; returns (B, h_q, h_kv, d, dtype code, device index)."""
+    for name, t in zip(_NAMES, (q, k_cache, v_cache, seqlens)):
         if not isinstance(t, torch.Tensor) or not t.is_cuda:
             raise ValueError(f"{name} must be a CUDA tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
-    if not (q.device == k_cache.device == v_cache.device == seqlens.device):
+    idx = q.get_device()
+    if not (k_cache.get_device() == v_cache.get_device() == seqlens.get_device() == idx):
         raise ValueError("all tensors must be on one device")
-    if q.dim() != 3 or k_cache.dim() != 3 or v_cache.shape != k_cache.shape:
+    qs, ks = q.shape, k_cache.shape
+    if len(qs) != 3 or len(ks) != 3 or v_cache.shape != ks:
         raise ValueError("q must be [B, h_q, d]; k_cache, v_cache [rows, h_kv, d]")
-    if q.dtype != k_cache.dtype or q.dtype != v_cache.dtype:
+    dt = q.dtype
+    if dt != k_cache.dtype or dt != v_cache.dtype:
         raise ValueError("q, k_cache and v_cache must share one dtype")
-    if seqlens.dtype != torch.int32 or seqlens.dim() != 1 or seqlens.shape[0] != q.shape[0]:
+    if seqlens.dtype != torch.int32 or seqlens.dim() != 1 or seqlens.shape[0] != qs[0]:
         raise ValueError("seqlens must be int32 [B]")
-    if q.shape[2] != k_cache.shape[2]:
+    if qs[2] != ks[2]:
         raise ValueError("head dims differ")
-    B, h_q, d = q.shape
-    return B, h_q, k_cache.shape[1], d, _dtype_code(q)
+    if dt == torch.bfloat16:
+        code = BF16
+    elif dt == torch.float32:
+        code = F32
+    else:
+        raise TypeError(f"q/k/v must be bf16 or fp32, got {dt}")
+    return qs[0], qs[1], ks[1], qs[2], code, idx
 
 
 _dummies: dict = {}
@@ -173,6 +204,24 @@ def _out(out, shape, device):
     return out
 
 
+def _out_idx(out, shape, idx: int):
+    """_out for the decode entry points (device given as an index)."""
+    if out is None:
+        return torch.empty(shape, dtype=torch.float32, device=torch.device("cuda", idx))
+    if (out.dtype != torch.float32 or out.shape != shape or not out.is_contiguous()
+            or out.get_device() != idx):
+        raise ValueError(f"out must be contiguous fp32 {tuple(shape)} on the inputs' device")
+    return out
+
+
+def _ws(workspace, idx: int, need_fn, *shape):
+    """(pointer, bytes) of the caller's workspace, or of the binding's own
+    grow-only one sized by need_fn(*shape)."""
+    if workspace is None:
+        workspace = _workspace(torch.device("cuda", idx), need_fn(*shape))
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
 def workspace_size(B, h_q, h_kv, d, n_splits) -> int:
     return _ws_size(B, h_q, h_kv, d, n_splits)
 
@@ -184,16 +233,12 @@ def chunked_workspace_size(B, h_q, h_kv, d, chunk_len, max_seqlen) -> int:
 def gqa_decode_attn(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, out=None,
                     workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Fused split-KV decode attention (split by count); returns fp32 [B, h_q, d]."""
-    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
-    out = _out(out, (B, h_q, d), q.device)
-    need = _ws_size(B, h_q, h_kv, d, n_splits)
-    if workspace is None:
-        workspace = _workspace(q.device, need)
-    with torch.cuda.device(q.device):
-        _check(_attn(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-                     out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
-                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                     _stream(q.device)), "gqa_decode_attn")
+    B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out_idx(out, (B, h_q, d), idx)
+    wp, wb = _ws(workspace, idx, _ws_size, B, h_q, h_kv, d, n_splits)
+    _check(_on(idx, _attn, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+               out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt, wp, wb,
+               _stream(idx)), "gqa_decode_attn")
     return out
 
 
@@ -206,12 +251,11 @@ def gqa_decode_attn_noalloc(q, k_cache, v_cache, seqlens, n_splits: int, scale=N
     GQADecodeError (ERR_WORKSPACE).  Calls share that array: keep them on one
     stream.  (Passing ``out=None`` still lets torch allocate the result here;
     pass ``out`` to avoid even that.)"""
-    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
-    out = _out(out, (B, h_q, d), q.device)
-    with torch.cuda.device(q.device):
-        _check(_attn_noalloc(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-                             out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
-                             _stream(q.device)), "gqa_decode_attn_noalloc")
+    B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out_idx(out, (B, h_q, d), idx)
+    _check(_on(idx, _attn_noalloc, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+               out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
+               _stream(idx)), "gqa_decode_attn_noalloc")
     return out
 
 
@@ -226,66 +270,56 @@ def gqa_decode_attn_append(q, k_new, v_new, k_cache, v_cache, seqlens, n_splits:
     for name, t in (("k_new", k_new), ("v_new", v_new)):
         if not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, h_kv, d) or t.dtype != q.dtype:
             raise ValueError(f"{name} must be a contiguous CUDA tensor [B, h_kv, d] of q's dtype")
-    _, h_q, _, _, dt = _inputs(q, k_cache.view(B * cap, h_kv, d), v_cache.view(B * cap, h_kv, d), seqlens)
-    out = _out(out, (B, h_q, d), q.device)
-    need = _ws_size(B, h_q, h_kv, d, n_splits)
-    if workspace is None:
-        workspace = _workspace(q.device, need)
-    with torch.cuda.device(q.device):
-        _check(_attn_append(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
-                            v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h_q, h_kv, d, cap,
-                            n_splits, _default_scale(d, scale), dt, workspace.data_ptr(),
-                            workspace.numel() * workspace.element_size(), _stream(q.device)),
-               "gqa_decode_attn_append")
+        if t.get_device() != q.get_device():
+            raise ValueError(f"{name} must be on q's device")
+    _, h_q, _, _, dt, idx = _inputs(q, k_cache.view(B * cap, h_kv, d), v_cache.view(B * cap, h_kv, d),
+                                    seqlens)
+    out = _out_idx(out, (B, h_q, d), idx)
+    wp, wb = _ws(workspace, idx, _ws_size, B, h_q, h_kv, d, n_splits)
+    _check(_on(idx, _attn_append, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_cache.data_ptr(),
+               v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h_q, h_kv, d, cap, n_splits,
+               _default_scale(d, scale), dt, wp, wb, _stream(idx)), "gqa_decode_attn_append")
     return out
 
 
 def gqa_decode_attn_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_seqlen: int,
                             scale=None, out=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Fused split-KV decode attention with fixed chunks (ragged batches)."""
-    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
-    out = _out(out, (B, h_q, d), q.device)
-    need = _ws_size_chunked(B, h_q, h_kv, d, chunk_len, max_seqlen)
-    if workspace is None:
-        workspace = _workspace(q.device, need)
-    with torch.cuda.device(q.device):
-        _check(_attn_chunked(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-                             out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
-                             _default_scale(d, scale), dt, workspace.data_ptr(),
-                             workspace.numel() * workspace.element_size(), _stream(q.device)),
-               "gqa_decode_attn_chunked")
+    B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
+    out = _out_idx(out, (B, h_q, d), idx)
+    wp, wb = _ws(workspace, idx, _ws_size_chunked, B, h_q, h_kv, d, chunk_len, max_seqlen)
+    _check(_on(idx, _attn_chunked, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+               out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
+               wp, wb, _stream(idx)), "gqa_decode_attn_chunked")
     return out
 
 
-def _triplets(B, h_q, n, d, device, m, l, o):
-    m = _out(m, (B, h_q, n), device)
-    l = _out(l, (B, h_q, n), device)
-    o = _out(o, (B, h_q, n, d), device)
+def _triplets(B, h_q, n, d, idx, m, l, o):
+    m = _out_idx(m, (B, h_q, n), idx)
+    l = _out_idx(l, (B, h_q, n), idx)
+    o = _out_idx(o, (B, h_q, n, d), idx)
     return m, l, o
 
 
 def gqa_decode_partial(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, m=None, l=None, o=None):
     """Per-split (m, l, o) triplets (split by count)."""
-    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
-    m, l, o = _triplets(B, h_q, n_splits, d, q.device, m, l, o)
-    with torch.cuda.device(q.device):
-        _check(_partial(q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-                        m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
-                        _default_scale(d, scale), dt, _stream(q.device)), "gqa_decode_partial")
+    B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
+    m, l, o = _triplets(B, h_q, n_splits, d, idx, m, l, o)
+    _check(_on(idx, _partial, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+               m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
+               _default_scale(d, scale), dt, _stream(idx)), "gqa_decode_partial")
     return m, l, o
 
 
 def gqa_decode_partial_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_seqlen: int,
                                scale=None, m=None, l=None, o=None):
     """Per-chunk (m, l, o) triplets; n_slots = max(1, ceil(max_seqlen / chunk_len))."""
-    B, h_q, h_kv, d, dt = _inputs(q, k_cache, v_cache, seqlens)
+    B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
     n = max(1, -(-max_seqlen // chunk_len)) if chunk_len > 0 and max_seqlen >= 0 else 1
-    m, l, o = _triplets(B, h_q, n, d, q.device, m, l, o)
-    with torch.cuda.device(q.device):
-        _check(_partial_chunked(q.data_ptr(), _ptr(k_cache), _ptr(v_cache),
-                                seqlens.data_ptr(), m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q,
-                                h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
-                                _stream(q.device)), "gqa_decode_partial_chunked")
+    m, l, o = _triplets(B, h_q, n, d, idx, m, l, o)
+    _check(_on(idx, _partial_chunked, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
+               m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
+               _default_scale(d, scale), dt, _stream(idx)), "gqa_decode_partial_chunked")
     return m, l, o
 
 
@@ -294,15 +328,17 @@ def mlo_merge(m, l, o, out=None) -> torch.Tensor:
     for name, t in (("m", m), ("l", l), ("o", o)):
         if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    idx = m.get_device()
+    if l.get_device() != idx or o.get_device() != idx:
+        raise ValueError("m, l and o must be on one device")
     n, d = o.shape[-2], o.shape[-1]
     lead = tuple(m.shape[:-1])
     if tuple(m.shape) != lead + (n,) or tuple(l.shape) != lead + (n,) or tuple(o.shape) != lead + (n, d):
         raise ValueError("shapes: m, l [..., n]; o [..., n, d]")
     rows = int(math.prod(lead))
-    out = _out(out, lead + (d,), m.device)
-    with torch.cuda.device(m.device):
-        _check(_merge(m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
-                      _stream(m.device)), "mlo_merge")
+    out = _out_idx(out, torch.Size(lead + (d,)), idx)
+    _check(_on(idx, _merge, m.data_ptr(), l.data_ptr(), o.data_ptr(), out.data_ptr(), rows, n, d,
+               _stream(idx)), "mlo_merge")
     return out
 
 

@@ -89,6 +89,38 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int h_kv, int D) {
   return r == CUDA_SUCCESS;
 }
 
+// Decode cache maps of recent calls.  A map is a pure function of (base
+// address, h_kv, D) -- the row extent is the fixed clip bound above -- so a
+// cached map is exactly what encoding again would give; the cache only saves
+// the driver call on the launch path.  Per host thread, a few entries
+// replaced round-robin.
+struct CacheMapEntry {
+  const void* base;
+  int h_kv, D;
+  CUtensorMap map;
+};
+
+bool cached_cache_map(CUtensorMap* map, const void* base, int h_kv, int D) {
+  constexpr int kEntries = 16;
+  thread_local CacheMapEntry entries[kEntries] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kEntries; ++i) {
+    const CacheMapEntry& e = entries[i];
+    if (e.base == base && e.h_kv == h_kv && e.D == D) {
+      *map = e.map;
+      return true;
+    }
+  }
+  if (!encode_cache_map(map, base, h_kv, D)) return false;
+  CacheMapEntry& e = entries[next];
+  next = (next + 1) % kEntries;
+  e.base = base;
+  e.h_kv = h_kv;
+  e.D = D;
+  e.map = *map;
+  return true;
+}
+
 // One-time (per device) opt-in to large dynamic shared memory for a kernel.
 template <typename K>
 int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done) {
@@ -152,7 +184,7 @@ int launch_tc(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
   auto kern = decode_tc_bf16<D, NT, NW, NS, MODE>;
   if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
   CUtensorMap kmap, vmap;
-  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
+  if (!cached_cache_map(&kmap, a.k, a.h_kv, D) || !cached_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
   return launch_pdl(kern, grid, dim3(NW * 32), smem, st, kmap, vmap, a);
 }
@@ -214,7 +246,7 @@ int launch_persist(const DecodeArgs& a, cudaStream_t st) {
   const long long units_max = (long long)a.n_slots * a.h_kv * a.n_hb * a.B;
   const int ctas = (int)(units_max < (long long)sms * occ ? units_max : (long long)sms * occ);
   CUtensorMap kmap, vmap;
-  if (!encode_cache_map(&kmap, a.k, a.h_kv, D) || !encode_cache_map(&vmap, a.v, a.h_kv, D))
+  if (!cached_cache_map(&kmap, a.k, a.h_kv, D) || !cached_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
   if (int rc = launch_pdl(kern, dim3(ctas), dim3(NW * 32), smem, st, kmap, vmap, a)) return rc;
   const long long rows = (long long)a.B * a.h_q;
