@@ -222,6 +222,23 @@ int fused_plan(long long units, int D) {
   return kPlanManyWaves;
 }
 
+// The row merge of the fused paths that store split triplets first: one warp
+// per row over the row's non-empty splits (programmatic dependent launch).
+int launch_merge_rows(const DecodeArgs& a, int D, cudaStream_t st) {
+  const long long rows = (long long)a.B * a.h_q;
+  const dim3 grid((unsigned)((rows + 3) / 4));
+  if (D == 128) return launch_pdl(merge_rows_kernel<4>, grid, dim3(128), 0, st, a, D);
+  return launch_pdl(merge_rows_kernel<2>, grid, dim3(128), 0, st, a, D);
+}
+
+// One-wave plan: whether the splits' triplets are merged by a second kernel
+// rather than by the CTA that finishes a group last.  That CTA merges the
+// group's G rows alone, at the very end of the call: with one row (G = 1) it
+// is quicker than a second launch, with G >= 8 rows the second kernel, which
+// spreads the rows over many CTAs, is (measured on B200: 16.3 against
+// 16.8 us at G = 1, 49.6 against 47.4 us at G = 8).
+inline bool one_wave_merge_kernel(int G) { return G >= 8; }
+
 // Fused bf16: persistent CTAs over the non-empty splits (as many as fit on
 // the GPU at once), then the row merge.  Both launches overlap their
 // predecessor's tail (programmatic dependent launch).
@@ -249,9 +266,7 @@ int launch_persist(const DecodeArgs& a, cudaStream_t st) {
   if (!cached_cache_map(&kmap, a.k, a.h_kv, D) || !cached_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
   if (int rc = launch_pdl(kern, dim3(ctas), dim3(NW * 32), smem, st, kmap, vmap, a)) return rc;
-  const long long rows = (long long)a.B * a.h_q;
-  return launch_pdl(merge_rows_kernel<D / 32>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st,
-                    a, D);
+  return launch_merge_rows(a, D, st);
 }
 
 template <int D, int HB, int MODE>
@@ -283,6 +298,15 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
       const long long units = (long long)grid.x * grid.y * grid.z;
       switch (fused_plan(units, D)) {
         case kPlanOneWave:
+          if (one_wave_merge_kernel(a.G)) {
+            int rc;
+            if (D == 128)
+              rc = wide ? launch_tc<128, 2, kPartial>(a, grid, st) : launch_tc<128, 1, kPartial>(a, grid, st);
+            else
+              rc = wide ? launch_tc<64, 2, kPartial>(a, grid, st) : launch_tc<64, 1, kPartial>(a, grid, st);
+            if (rc) return rc;
+            return launch_merge_rows(a, D, st);
+          }
           if (D == 128)
             return wide ? launch_tc<128, 2, kFused>(a, grid, st) : launch_tc<128, 1, kFused>(a, grid, st);
           return wide ? launch_tc<64, 2, kFused>(a, grid, st) : launch_tc<64, 1, kFused>(a, grid, st);
@@ -687,15 +711,11 @@ int gqa_decode_attn_noalloc(const void* q, const void* k_cache, const void* v_ca
   void* scratch = nullptr;
   if (int rc = noalloc_scratch(&scratch)) return rc;
   // The array keeps whatever the previous call left; the tickets must start
-  // at zero, so clear this call's part of the ticket area first.  The
-  // persistent plan merges in its second kernel and reads no ticket, so a
-  // call that takes it needs no clearing.
-  bool uses_tickets = true;
-  if (dtype == GQA_BF16) {
-    const int G = h_q / h_kv, hb = tc_heads_per_cta(G);
-    const long long units = (long long)s.n_slots * h_kv * ((G + hb - 1) / hb) * B;
-    uses_tickets = fused_plan(units, d_head) != kPlanPersistent;
-  }
+  // at zero, so clear this call's part of the ticket area first.  A call
+  // that merges in a second kernel (two launches) reads no ticket and needs
+  // no clearing.
+  const bool uses_tickets =
+      gqa_decode_launches_per_call(B, h_q, h_kv, d_head, s.n_slots, dtype) != 2;
   if (uses_tickets &&
       cudaMemsetAsync(scratch, 0, n_tickets(s) * sizeof(int), as_stream(stream)) != cudaSuccess) {
     cudaGetLastError();
@@ -805,7 +825,7 @@ int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slo
   const long long units = (long long)n_slots * h_kv * ((G + hb - 1) / hb) * B;
   const int plan = fused_plan(units, d_head);
   if (plan < 0) return -GQA_ERR_CUDA;
-  return plan == kPlanPersistent ? 2 : 1;
+  return (plan == kPlanPersistent || (plan == kPlanOneWave && one_wave_merge_kernel(G))) ? 2 : 1;
 }
 
 int gqa_prefill_attn(const void* q, const void* k, const void* v, const int32_t* seqlens,

@@ -139,7 +139,7 @@ GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_ca
  * address (cudaGetSymbolAddress) with that device current; make that first
  * call before any stream capture.  Every call clears the tickets it uses
  * (one cudaMemsetAsync on the stream) and then runs the fused kernels; a call
- * that takes the persistent plan (gqa_decode_launches_per_call == 2) reads no
+ * that merges in a second kernel (gqa_decode_launches_per_call == 2) reads no
  * ticket and skips the clearing.  Nothing is allocated or freed.  All calls on a device share that device's one array,
  * which keeps the last call's contents: calls that overlap on the GPU (for
  * instance on two streams) race and corrupt each other's results, so order
@@ -250,9 +250,11 @@ GQA_API int gqa_decode_auto_splits(int B, int h_q, int h_kv, int d_head, int max
 /*
  * Number of kernels one fused call (gqa_decode_attn / _chunked / _noalloc)
  * launches on the current device for this shape (n_slots = n_splits, or
- * ceil(max_seqlen / chunk_len) when chunked): 1, or 2 when the persistent
- * decode kernel plus its row merge is chosen.  0 for B == 0; a negative
- * gqa_status on bad arguments.
+ * ceil(max_seqlen / chunk_len) when chunked): 1 when the CTA that finishes a
+ * group's splits last merges them, or 2 when the splits' triplets are merged
+ * by a second kernel -- the persistent decode kernel, and the one-wave grid
+ * of groups of 8 or more query heads.  0 for B == 0; a negative gqa_status
+ * on bad arguments.
  */
 GQA_API int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slots,
                                          int dtype);

@@ -3,7 +3,10 @@
 The plan follows from the grid size (units = splits x kv heads x head blocks
 x batch) against R, the per-split CTAs resident at once (2 per SM at d = 128,
 4 at d = 64): one wave (units <= R), persistent (R < units <= 4R), many waves
-(units > 4R).  The shapes below land in each plan on a 148-SM B200.
+(units > 4R).  One launch merges by ticket inside the kernel; two launches
+store the split triplets and merge them in a second kernel (the persistent
+plan, and the one-wave plan for groups of 8 or more query heads).  The
+shapes below land in each plan on a 148-SM B200.
 """
 import numpy as np
 import pytest
@@ -36,7 +39,8 @@ def _check(got, w):
 
 # (B, h_q, h_kv, d, seqlens, n_splits, launches expected on 148 SMs)
 CASES = [
-    (3, 16, 2, 128, [100, 0, 2000], 4, 1),                   # one wave
+    (3, 16, 2, 128, [100, 0, 2000], 4, 2),                   # one wave, merge kernel (G = 8)
+    (3, 16, 4, 128, [100, 0, 2000], 4, 1),                   # one wave, ticket merge (G = 4)
     (4, 64, 8, 128, [0, 1, 17, 3000], 16, 2),                 # persistent; empty and 1-key sequences
     (4, 64, 4, 128, [900, 2, 0, 4000], 32, 2),                # persistent, 16-head blocks
     (6, 64, 8, 64, [300, 40, 5000, 1, 77, 1200], 16, 2),      # persistent, d = 64 (R = 4 per SM)
@@ -97,7 +101,8 @@ def test_auto_split_count(gk, case):
     B, hq, hkv, d, S = case
     n = gk.auto_splits(B, hq, hkv, d)
     assert 1 <= n <= 1024
-    assert gk.launches_per_call(B, hq, hkv, d, n) == 1       # one wave: one launch
+    # one wave: the ticket merge (one launch), or a merge kernel for G >= 8
+    assert gk.launches_per_call(B, hq, hkv, d, n) == (2 if hq // hkv >= 8 else 1)
     assert gk.auto_splits(B, hq, hkv, d, max_seqlen=300) <= 2  # >= 256 keys per split
     w = random_case(B, hq, hkv, d, [S] * B if B > 1 else [S], dtype="bf16", seed=B + S)
     q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()

@@ -8,8 +8,9 @@ call it through the C ABI (via the ctypes binding) and check it against the
 fp64 oracle and against the workspace entry point, gqa_decode_attn, on two
 calls in a row -- the second call finds the array as the first one left it.
 The shapes cover both kinds of fused plan: the single-launch plans that
-merge through tickets in the array, and the persistent plan whose two
-kernels keep their triplets there.  This file is collected last so that a
+merge through tickets in the array, and the two-launch plans (persistent,
+or one wave of groups of 8 query heads) whose kernels keep their triplets
+there.  This file is collected last so that a
 run stopping at the first failure has run every other test.
 """
 import numpy as np
@@ -47,7 +48,8 @@ def _oracle(w):
 
 # (B, h_q, h_kv, d, seqlens, n_splits, dtype, launches per call on a 148-SM B200)
 CASES = [
-    (3, 64, 8, 128, [3000, 17, 900], 8, "bf16", 1),          # one wave, ticket merge
+    (3, 32, 8, 128, [3000, 17, 900], 8, "bf16", 1),          # one wave, ticket merge (G = 4)
+    (3, 64, 8, 128, [3000, 17, 900], 8, "bf16", 2),          # one wave, merge kernel (G = 8)
     (3, 64, 8, 128, [3000, 17, 900], 8, "f32", 1),
     (4, 64, 8, 128, [0, 1, 17, 3000], 16, "bf16", 2),        # persistent kernel + row merge
     (6, 64, 8, 128, [5, 0, 700, 33, 4096, 16], 32, "bf16", 1),  # many waves, ticket merge
