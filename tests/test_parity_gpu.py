@@ -4,7 +4,15 @@ Tolerances (elementwise, allclose convention):
     bf16 inputs: |gpu - oracle| <= 2e-3 + 1e-2 * |oracle|
     fp32 inputs: |gpu - oracle| <= 1e-5 + 1e-5 * |oracle|
 Triplets are compared as m (absolute, scaled by max(1, |m|)), l (relative)
-and the split's normalised output o / l (the tolerance above).
+and the split's normalised output o / l (the tolerance above).  The method's
+pages fix no triplet tolerance; the bounds below are readings from fp32
+rounding: a logit is an fp32 sum of d = 128 exact bf16 (or fp32) products,
+off by at most about d * 2^-24 of its magnitude, so m is within 1e-5 of
+max(1, |m|); l sums up to a few thousand fp32 exponentials (each off by
+twice the logit error plus the exp2 rounding) in short sequential runs and a
+shuffle tree, so its relative error stays below 1e-4 for bf16 inputs (and
+1e-5 for the fp32 path).  Measured worst cases on B200 over the workloads and
+edge cases: 4.9e-7 (m) and 1.3e-6 (l).
 """
 import zlib
 
@@ -19,8 +27,8 @@ from workloads import CONFIGS, random_case, scaled
 pytestmark = pytest.mark.gpu
 
 TOL = {"bf16": (2e-3, 1e-2), "f32": (1e-5, 1e-5)}
-M_TOL = {"bf16": 1e-4, "f32": 1e-5}
-L_RTOL = {"bf16": 4e-3, "f32": 1e-5}
+M_TOL = {"bf16": 1e-5, "f32": 1e-5}
+L_RTOL = {"bf16": 1e-4, "f32": 1e-5}
 
 
 @pytest.fixture(scope="module")

@@ -1,9 +1,10 @@
 """Causal prefill (gqa_prefill_attn, tcgen05 kernel) against the oracle.
 
-Every output of the small cases is compared element by element; the
-full-size workloads are compared on sampled (sequence, head, position) rows
-that include each 128-row tile's first and last rows and each sequence's
-first and last positions.  Bound: |e| <= 2e-3 + 1e-2 |ref| (bf16 inputs).
+Every output of the small cases and of the two full-size workloads is
+compared element by element; the 32k-token prompt is compared on sampled
+(sequence, head, position) rows that include each 128-row tile's first and
+last rows and each sequence's first and last positions.  Bound:
+|e| <= 2e-3 + 1e-2 |ref| (bf16 inputs).
 """
 import numpy as np
 import pytest
@@ -117,17 +118,14 @@ def _sample_items(seqlens, h_q, n, seed):
 
 
 @pytest.mark.parametrize("name", ["llama70b_prefill2k", "prefill_ragged"])
-def test_prefill_full_size_sampled(gk, name):
+def test_prefill_full_size_every_row(gk, name):
+    """The two prefill workloads at full size, every output element against
+    the oracle (a full fp64 pass takes seconds on the host's cores)."""
     w = generate_prefill(name)
     got = _run(gk, w)
     assert gk.get_status() == 0
-    sl = w.seqlens.tolist()
-    items = _sample_items(sl, w.h_q, 1500, seed=7)
-    ref = oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale, items=items)
-    off = np.concatenate([[0], np.cumsum(sl)])
-    rows = np.array([(off[b] + i) for b, h, i in items])
-    heads = np.array([h for b, h, i in items])
-    _assert_close(got[rows, heads], ref)
+    ref = oracle.prefill(w.q, w.k, w.v, w.seqlens, w.h_q, w.h_kv, w.scale)
+    _assert_close(got.reshape(-1, w.d), ref)
 
 
 def test_prefill_long_prompt_sampled(gk):
