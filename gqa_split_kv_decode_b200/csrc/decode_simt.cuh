@@ -2,9 +2,10 @@
 //
 // fp32 inputs must not go through TF32 or bf16 tensor-core products (the fp32
 // tolerance is 1e-5), so this path uses plain FMA.  It serves the small fp32
-// workloads, which are launch-bound: a warp streams one key row per step with
-// 16-byte (D = 128) or 8-byte (D = 64) loads per lane, all HB query heads of
-// the block reuse that row, and the online softmax is kept per warp in base 2.
+// workloads, which are latency-bound: a warp streams its keys in batches,
+// each key row read with 16-byte (D = 128) or 8-byte (D = 64) loads per lane,
+// all HB query heads of the block reuse each row, and the online softmax is
+// kept per warp in base 2.
 #pragma once
 
 #include "split_merge.cuh"
@@ -56,37 +57,73 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
   }
 
   const size_t new_base = ((size_t)b * a.h_kv + g) * D + lane * PER;
-  for (int j = sp.lo + warp; j < sp.hi; j += NW) {
-    // key j comes from the cache, or is the appended token (key number cached_hi)
-    const bool fresh = sp.has_new && j == sp.cached_hi;
-    const size_t base = fresh ? new_base : ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
-    const float* ksrc = fresh ? static_cast<const float*>(a.k_new) : kp;
-    const float* vsrc = fresh ? static_cast<const float*>(a.v_new) : vp;
-    float kr[PER], vr[PER];
-    if constexpr (PER == 4) {
-      const float4 k4 = __ldg(reinterpret_cast<const float4*>(ksrc + base));
-      const float4 v4 = __ldg(reinterpret_cast<const float4*>(vsrc + base));
-      kr[0] = k4.x; kr[1] = k4.y; kr[2] = k4.z; kr[3] = k4.w;
-      vr[0] = v4.x; vr[1] = v4.y; vr[2] = v4.z; vr[3] = v4.w;
-    } else {
-      const float2 k2 = __ldg(reinterpret_cast<const float2*>(ksrc + base));
-      const float2 v2 = __ldg(reinterpret_cast<const float2*>(vsrc + base));
-      kr[0] = k2.x; kr[1] = k2.y;
-      vr[0] = v2.x; vr[1] = v2.y;
+  // Keys in batches of U per warp (keys j0, j0 + NW, ..., j0 + (U-1) NW): the
+  // batch's K and V rows are requested together, so a warp waits one memory
+  // round trip per batch rather than per key, and the batch's logits share
+  // one max update.
+  constexpr int U = (HB * PER <= 16) ? 8 : 4;
+  for (int j0 = sp.lo + warp; j0 < sp.hi; j0 += NW * U) {
+    float kr[U][PER], vr[U][PER];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * NW;
+      if (j < sp.hi) {
+        // key j comes from the cache, or is the appended token (key number cached_hi)
+        const bool fresh = sp.has_new && j == sp.cached_hi;
+        const size_t base = fresh ? new_base : ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
+        const float* ksrc = fresh ? static_cast<const float*>(a.k_new) : kp;
+        const float* vsrc = fresh ? static_cast<const float*>(a.v_new) : vp;
+        if constexpr (PER == 4) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4*>(ksrc + base));
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(vsrc + base));
+          kr[u][0] = k4.x; kr[u][1] = k4.y; kr[u][2] = k4.z; kr[u][3] = k4.w;
+          vr[u][0] = v4.x; vr[u][1] = v4.y; vr[u][2] = v4.z; vr[u][3] = v4.w;
+        } else {
+          const float2 k2 = __ldg(reinterpret_cast<const float2*>(ksrc + base));
+          const float2 v2 = __ldg(reinterpret_cast<const float2*>(vsrc + base));
+          kr[u][0] = k2.x; kr[u][1] = k2.y;
+          vr[u][0] = v2.x; vr[u][1] = v2.y;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) kr[u][e] = vr[u][e] = 0.f;
+      }
     }
 #pragma unroll
     for (int hh = 0; hh < HB; ++hh) {
       if (hb * HB + hh >= a.G) break;
-      float part = 0.f;
+      float s[U];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) part = fmaf(qr[hh][e], kr[e], part);
-      const float s = warp_sum(part) * a.scale_log2;
-      const float m_new = fmaxf(m_run[hh], s);
-      const float alpha = exp2f(m_run[hh] - m_new);  // 0 on the first key
-      const float p = exp2f(s - m_new);
-      l_run[hh] = fmaf(l_run[hh], alpha, p);
+      for (int u = 0; u < U; ++u) {
+        float part = 0.f;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) o_acc[hh][e] = fmaf(o_acc[hh][e], alpha, p * vr[e]);
+        for (int e = 0; e < PER; ++e) part = fmaf(qr[hh][e], kr[u][e], part);
+        s[u] = part;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(kFull, s[u], o);
+      float mb = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        s[u] = (j0 + u * NW < sp.hi) ? s[u] * a.scale_log2 : -INFINITY;
+        mb = fmaxf(mb, s[u]);
+      }
+      // key j0 is in the range, so the batch max is finite
+      const float m_new = fmaxf(m_run[hh], mb);
+      const float alpha = exp2f(m_run[hh] - m_new);  // 0 on the first batch
+      float psum = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o_acc[hh][e] *= alpha;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float p = exp2f(s[u] - m_new);  // 0 past the range
+        psum += p;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) o_acc[hh][e] = fmaf(p, vr[u][e], o_acc[hh][e]);
+      }
+      l_run[hh] = fmaf(l_run[hh], alpha, psum);
       m_run[hh] = m_new;
     }
   }
