@@ -53,6 +53,10 @@ def test_decode_bench_line():
     assert d["config"]["seed"] == workloads.CONFIGS["llama70b"].seed
     pm = d["partial_merge"]
     assert pm["us_per_call"] > 0 and pm["steps"] == 200
+    # the same K steps as direct calls: the graph replay removes host launch
+    # work only, so the two agree closely
+    dc = d["direct_calls"]
+    assert 0.5 < dc["ms_per_step"] / d["ms_per_step"] < 2.0
     # every other workload, timed the same way
     assert sorted(d["per_config"]) == sorted(n for n in workloads.CONFIGS if n != "llama70b")
     for name, e in d["per_config"].items():
