@@ -322,8 +322,9 @@ class DecodeRig:
             self.n_slots = cfg.n_splits
             ws = gk.workspace_size(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, cfg.n_splits)
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=device)
-        self.launches = gk.launches_per_call(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, self.n_slots,
-                                             gk.BF16 if cfg.dtype == "bf16" else gk.F32, device)
+        dt = gk.BF16 if cfg.dtype == "bf16" else gk.F32
+        self.launches = gk.launches_per_call(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, self.n_slots, dt, device)
+        self.plan = gk.fused_plan(cfg.B, cfg.h_q, cfg.h_kv, cfg.d, self.n_slots, dt, device)
         shape = (cfg.B, cfg.h_q, self.n_slots)
         self.m = torch.empty(shape, dtype=torch.float32, device=device)
         self.l = torch.empty(shape, dtype=torch.float32, device=device)
@@ -349,9 +350,13 @@ class DecodeRig:
         self.gk.mlo_merge(self.m, self.l, self.o, out=self.out)
 
     def kernel_name(self) -> str:
-        if self.cfg.dtype != "bf16":
-            return "decode_simt_f32 (fused)"
-        return "decode_tc_bf16_persist + merge_rows_kernel" if self.launches == 2 else "decode_tc_bf16 (fused)"
+        if self.plan == "simt":
+            return "decode_simt_f32 (fused, ticket merge)"
+        if self.plan == "persistent":
+            return "decode_tc_bf16_persist + merge_rows_kernel"
+        if self.launches == 2:
+            return f"decode_tc_bf16 ({self.plan}) + merge_rows_kernel"
+        return f"decode_tc_bf16 ({self.plan}, ticket merge)"
 
 
 def upload_graph(g, stream) -> bool:

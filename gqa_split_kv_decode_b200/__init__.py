@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "gqa_decode_attn", "gqa_decode_attn_noalloc", "gqa_decode_attn_append", "gqa_decode_attn_chunked", "gqa_decode_partial",
     "gqa_decode_partial_chunked", "mlo_merge", "workspace_size", "chunked_workspace_size",
-    "gqa_prefill_attn", "mlo_merge_ranked", "mlo_merge_ranked_raw", "get_status", "auto_splits", "launches_per_call", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
+    "gqa_prefill_attn", "mlo_merge_ranked", "mlo_merge_ranked_raw", "get_status", "auto_splits", "launches_per_call", "fused_plan", "set_wait_timeout_ns", "selftest_wait_timeout", "release", "version",
     "checked_build", "bounds_report", "selftest_bounds",
     "GQADecodeError", "LIB_PATH", "F32", "BF16",
 ]
@@ -76,6 +76,8 @@ _prefill = _sig("gqa_prefill_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci,
 _get_status = _sig("gqa_decode_get_status", _ci, _vp)
 _auto_splits = _sig("gqa_decode_auto_splits", _ci, _ci, _ci, _ci, _ci, _ci)
 _launches = _sig("gqa_decode_launches_per_call", _ci, _ci, _ci, _ci, _ci, _ci, _ci)
+_plan = _sig("gqa_decode_fused_plan", _ci, _ci, _ci, _ci, _ci, _ci, _ci)
+PLAN_NAMES = {0: "simt", 1: "one_wave", 2: "persistent", 3: "many_waves"}
 _set_timeout = _sig("gqa_decode_set_wait_timeout_ns", _ci, _ull)
 _selftest = _sig("gqa_decode_selftest_wait_timeout", _ci, _ull, _vp)
 _release = _sig("gqa_decode_release", _ci)
@@ -387,6 +389,17 @@ def launches_per_call(B, h_q, h_kv, d, n_slots, dtype=BF16, device=None) -> int:
     if n < 0:
         raise GQADecodeError(-n, "gqa_decode_launches_per_call")
     return n
+
+
+def fused_plan(B, h_q, h_kv, d, n_slots, dtype=BF16, device=None) -> str:
+    """Launch plan of a fused call for this shape on ``device``: "simt" (fp32),
+    "one_wave", "persistent" or "many_waves"."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(device):
+        n = _plan(B, h_q, h_kv, d, n_slots, dtype)
+    if n < 0:
+        raise GQADecodeError(-n, "gqa_decode_fused_plan")
+    return PLAN_NAMES[n]
 
 
 def get_status(device=None) -> int:

@@ -828,6 +828,21 @@ int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slo
   return (plan == kPlanPersistent || (plan == kPlanOneWave && one_wave_merge_kernel(G))) ? 2 : 1;
 }
 
+int gqa_decode_fused_plan(int B, int h_q, int h_kv, int d_head, int n_slots, int dtype) {
+  const Shape s = split_shape(B, h_q, h_kv, d_head, n_slots, 1.f, dtype);
+  if (check_shape(s) || B == 0) return -GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_BF16) return GQA_PLAN_SIMT;
+  const int G = h_q / h_kv;
+  const int hb = tc_heads_per_cta(G);
+  const long long units = (long long)n_slots * h_kv * ((G + hb - 1) / hb) * B;
+  switch (fused_plan(units, d_head)) {
+    case kPlanOneWave: return GQA_PLAN_ONE_WAVE;
+    case kPlanPersistent: return GQA_PLAN_PERSISTENT;
+    case kPlanManyWaves: return GQA_PLAN_MANY_WAVES;
+    default: return -GQA_ERR_CUDA;
+  }
+}
+
 int gqa_prefill_attn(const void* q, const void* k, const void* v, const int32_t* seqlens,
                      float* out, int B, int total_rows, int max_seqlen, int h_q, int h_kv,
                      int d_head, float scale, int dtype, void* stream) {

@@ -140,7 +140,8 @@ GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_ca
  * call before any stream capture.  Every call clears the tickets it uses
  * (one cudaMemsetAsync on the stream) and then runs the fused kernels; a call
  * that merges in a second kernel (gqa_decode_launches_per_call == 2) reads no
- * ticket and skips the clearing.  Nothing is allocated or freed.  All calls on a device share that device's one array,
+ * ticket and skips the clearing.  Nothing is allocated or freed.  All calls
+ * on a device share that device's one array,
  * which keeps the last call's contents: calls that overlap on the GPU (for
  * instance on two streams) race and corrupt each other's results, so order
  * them on one stream.
@@ -258,6 +259,23 @@ GQA_API int gqa_decode_auto_splits(int B, int h_q, int h_kv, int d_head, int max
  */
 GQA_API int gqa_decode_launches_per_call(int B, int h_q, int h_kv, int d_head, int n_slots,
                                          int dtype);
+
+/*
+ * The launch plan one fused call takes on the current device for this shape
+ * (arguments as for gqa_decode_launches_per_call):
+ *   GQA_PLAN_SIMT        fp32: one CUDA-core kernel per (split, kv head, b);
+ *   GQA_PLAN_ONE_WAVE    bf16, every split CTA resident at once: one
+ *                        tensor-core kernel, merged by ticket (groups of
+ *                        fewer than 8 query heads) or by a second kernel;
+ *   GQA_PLAN_PERSISTENT  bf16, up to four times that many splits: persistent
+ *                        CTAs over the splits, then the row-merge kernel;
+ *   GQA_PLAN_MANY_WAVES  bf16, more: the per-split kernel with two stages per
+ *                        warp, merged by ticket.
+ * Returns the plan (>= 0), or a negative gqa_status on bad arguments
+ * (-GQA_ERR_INVALID_ARG also for B == 0, which launches nothing).
+ */
+enum { GQA_PLAN_SIMT = 0, GQA_PLAN_ONE_WAVE = 1, GQA_PLAN_PERSISTENT = 2, GQA_PLAN_MANY_WAVES = 3 };
+GQA_API int gqa_decode_fused_plan(int B, int h_q, int h_kv, int d_head, int n_slots, int dtype);
 
 /*
  * Synchronises `stream`, then reads and clears this device's status word.

@@ -154,6 +154,10 @@ def test_launch_count_query_without_a_gpu(lib):
     assert lib.gqa_decode_launches_per_call(0, 8, 2, 128, 4, 1) == 0      # empty batch
     assert lib.gqa_decode_launches_per_call(2, 8, 2, 128, 4, 0) == 1      # fp32: one kernel
     assert lib.gqa_decode_launches_per_call(2, 6, 4, 128, 4, 1) == -INVALID
+    lib.gqa_decode_fused_plan.argtypes = [ctypes.c_int] * 6
+    assert lib.gqa_decode_fused_plan(2, 8, 2, 128, 4, 0) == 0          # fp32: the CUDA-core kernel
+    assert lib.gqa_decode_fused_plan(2, 6, 4, 128, 4, 1) == -INVALID    # h_q not a multiple of h_kv
+    assert lib.gqa_decode_fused_plan(0, 8, 2, 128, 4, 1) == -INVALID    # nothing to plan
 
 
 @pytest.mark.parametrize("kw,expect", [

@@ -37,25 +37,27 @@ def _check(got, w):
     assert (err <= bound).all(), float((err - bound).max())
 
 
-# (B, h_q, h_kv, d, seqlens, n_splits, launches expected on 148 SMs)
+# (B, h_q, h_kv, d, seqlens, n_splits, plan and launches expected on 148 SMs)
 CASES = [
-    (3, 16, 2, 128, [100, 0, 2000], 4, 2),                   # one wave, merge kernel (G = 8)
-    (3, 16, 4, 128, [100, 0, 2000], 4, 1),                   # one wave, ticket merge (G = 4)
-    (4, 64, 8, 128, [0, 1, 17, 3000], 16, 2),                 # persistent; empty and 1-key sequences
-    (4, 64, 4, 128, [900, 2, 0, 4000], 32, 2),                # persistent, 16-head blocks
-    (6, 64, 8, 64, [300, 40, 5000, 1, 77, 1200], 16, 2),      # persistent, d = 64 (R = 4 per SM)
-    (6, 64, 8, 128, [5, 0, 700, 33, 4096, 16], 32, 1),        # many waves
-    (2, 96, 2, 128, [2500, 300], 200, 1),                     # many waves, 3 head blocks of 16
+    (3, 16, 2, 128, [100, 0, 2000], 4, "one_wave", 2),          # merge kernel (G = 8)
+    (3, 16, 4, 128, [100, 0, 2000], 4, "one_wave", 1),          # ticket merge (G = 4)
+    (4, 64, 8, 128, [0, 1, 17, 3000], 16, "persistent", 2),     # empty and 1-key sequences
+    (4, 64, 4, 128, [900, 2, 0, 4000], 32, "persistent", 2),    # 16-head blocks
+    (6, 64, 8, 64, [300, 40, 5000, 1, 77, 1200], 16, "persistent", 2),  # d = 64 (R = 4 per SM)
+    (6, 64, 8, 128, [5, 0, 700, 33, 4096, 16], 32, "many_waves", 1),
+    (2, 96, 2, 128, [2500, 300], 200, "many_waves", 1),         # 3 head blocks of 16
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}_hq{c[1]}_hkv{c[2]}_d{c[3]}_n{c[5]}" for c in CASES])
 def test_plan_matches_oracle(gk, case):
-    B, hq, hkv, d, seqlens, n, launches = case
+    B, hq, hkv, d, seqlens, n, plan, launches = case
     w = random_case(B, hq, hkv, d, seqlens, dtype="bf16", seed=sum(seqlens) % 997)
     c = w.cfg
     if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert gk.fused_plan(B, hq, hkv, d, n) == plan
         assert gk.launches_per_call(B, hq, hkv, d, n) == launches
+    assert gk.fused_plan(B, hq, hkv, d, n, dtype=gk.F32) == "simt"
     q, k, v, sl = w.q.cuda(), w.k.cuda(), w.v.cuda(), w.seqlens.cuda()
     for _ in range(2):  # twice: the second call reuses the workspace
         out = gk.gqa_decode_attn(q, k, v, sl, n, c.scale)
