@@ -1,5 +1,5 @@
-// Fused bf16 decode: persistent CTAs over the non-empty splits, then a merge
-// kernel over all rows.
+// bf16 decode over persistent CTAs: the fused call (then a merge kernel over
+// all rows) and, for grids of a few waves, the partial call.
 //
 // The per-split grid runs one CTA per (split, kv head, head block, b); when
 // there are more splits than resident CTAs the second wave starts cold and
@@ -169,7 +169,11 @@ constexpr int persist_dynamic_smem() {
   return NW * NS * TcShape<D>::kStageBytes + 2 * XSlot<D, NT>::kFloats * 4 + 1024;
 }
 
-template <int D, int NT, int NW, int NS>
+// PARTIAL: the call returns every split slot (gqa_decode_partial), so after
+// its units each CTA also writes the empty triplets (-inf, 0, 0) of the
+// slots past a sequence's non-empty splits, for a share of the (b, kv head /
+// head block) pairs.
+template <int D, int NT, int NW, int NS, bool PARTIAL>
 __global__ void __launch_bounds__(NW * 32)
     decode_tc_bf16_persist(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap vmap, const DecodeArgs a) {
@@ -360,6 +364,17 @@ __global__ void __launch_bounds__(NW * 32)
               }
             }
       }
+    }
+  }
+
+  if (PARTIAL) {
+    const long long pairs = (long long)a.B * H;
+    for (long long p = blockIdx.x; p < pairs; p += gridDim.x) {
+      const int b = (int)(p / H), gy = (int)(p % H);
+      int L;
+      const int n = active_splits(a, seq_keys(a, __ldg(a.seqlens + b)).total, L);
+      for (int slot = n; slot < a.n_slots; ++slot)
+        emit_empty_triplet<HB, D>(a, b, gy / a.n_hb, gy % a.n_hb, slot);
     }
   }
 }

@@ -242,13 +242,13 @@ inline bool one_wave_merge_kernel(int G) { return G >= 8; }
 // Fused bf16: persistent CTAs over the non-empty splits (as many as fit on
 // the GPU at once), then the row merge.  Both launches overlap their
 // predecessor's tail (programmatic dependent launch).
-template <int D, int NT>
+template <int D, int NT, bool PARTIAL>
 int launch_persist(const DecodeArgs& a, cudaStream_t st) {
   constexpr int NW = 4, NS = kTcStages;
   constexpr int smem = persist_dynamic_smem<D, NT, NW, NS>();
   static std::atomic<uint64_t> attr_done{0};
   static std::atomic<int> per_sm[kMaxDevices];
-  auto kern = decode_tc_bf16_persist<D, NT, NW, NS>;
+  auto kern = decode_tc_bf16_persist<D, NT, NW, NS, PARTIAL>;
   if (int rc = ensure_smem_attr(kern, smem, attr_done)) return rc;
   const int dev = current_device();
   const int sms = sm_count();
@@ -266,7 +266,7 @@ int launch_persist(const DecodeArgs& a, cudaStream_t st) {
   if (!cached_cache_map(&kmap, a.k, a.h_kv, D) || !cached_cache_map(&vmap, a.v, a.h_kv, D))
     return GQA_ERR_CUDA;
   if (int rc = launch_pdl(kern, dim3(ctas), dim3(NW * 32), smem, st, kmap, vmap, a)) return rc;
-  return launch_merge_rows(a, D, st);
+  return PARTIAL ? GQA_OK : launch_merge_rows(a, D, st);
 }
 
 template <int D, int HB, int MODE>
@@ -311,8 +311,9 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
             return wide ? launch_tc<128, 2, kFused>(a, grid, st) : launch_tc<128, 1, kFused>(a, grid, st);
           return wide ? launch_tc<64, 2, kFused>(a, grid, st) : launch_tc<64, 1, kFused>(a, grid, st);
         case kPlanPersistent:
-          if (D == 128) return wide ? launch_persist<128, 2>(a, st) : launch_persist<128, 1>(a, st);
-          return wide ? launch_persist<64, 2>(a, st) : launch_persist<64, 1>(a, st);
+          if (D == 128)
+            return wide ? launch_persist<128, 2, false>(a, st) : launch_persist<128, 1, false>(a, st);
+          return wide ? launch_persist<64, 2, false>(a, st) : launch_persist<64, 1, false>(a, st);
         case kPlanManyWaves:
           if (D == 128)
             return wide ? launch_tc<128, 2, kFused, 2>(a, grid, st)
@@ -321,6 +322,13 @@ int launch_decode(DecodeArgs a, int dtype, int D, cudaStream_t st) {
         default:
           return GQA_ERR_CUDA;
       }
+    }
+    // Partial call: a grid of a few waves runs on the persistent CTAs too
+    // (every split's triplet stored, empty ones included; no merge).
+    if (fused_plan((long long)grid.x * grid.y * grid.z, D) == kPlanPersistent) {
+      if (D == 128)
+        return wide ? launch_persist<128, 2, true>(a, st) : launch_persist<128, 1, true>(a, st);
+      return wide ? launch_persist<64, 2, true>(a, st) : launch_persist<64, 1, true>(a, st);
     }
     if (D == 128)
       return wide ? launch_tc<128, 2, kPartial>(a, grid, st) : launch_tc<128, 1, kPartial>(a, grid, st);
