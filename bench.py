@@ -394,6 +394,66 @@ def _timed_region(run, device, world):
     return s.elapsed_time(e), (h0, h1)
 
 
+def decode_loop_e2e(gk, cfg, w, rig, E: int, device, world: int):
+    """End to end as a decode loop runs: the KV cache stays resident in a
+    padded layout ([B][S_max + 1][h_kv][d]); every step copies q and the new
+    token's k and v in from pinned host memory, calls gqa_decode_attn_append
+    (which writes the token into the cache and attends over S_b + 1 keys) and
+    copies the result back.  seqlens is not advanced, so every step redoes
+    the same work (the new row is rewritten in place)."""
+    B, hkv, d = cfg.B, cfg.h_kv, cfg.d
+    sl = w.seqlens.tolist()
+    cap = max(sl) + 1
+    kp = torch.zeros((B, cap, hkv, d), dtype=w.k.dtype, device=device)
+    vp = torch.zeros_like(kp)
+    off = 0
+    for b, S in enumerate(sl):
+        kp[b, :S].copy_(w.k[off:off + S])
+        vp[b, :S].copy_(w.v[off:off + S])
+        off += S
+    gen = torch.Generator().manual_seed(cfg.seed + 7)
+    # q and the new token's k, v side by side in one pinned buffer, so a step
+    # moves its inputs with one host-to-device copy (views of one device buffer)
+    nq, nkv = B * cfg.h_q * d, B * hkv * d
+    hin = torch.empty(nq + 2 * nkv, dtype=w.q.dtype).pin_memory()
+    hin[:nq].copy_(w.q.reshape(-1))
+    hin[nq:].copy_(torch.randn(2 * nkv, generator=gen).to(w.q.dtype))
+    din = torch.empty_like(hin, device=device)
+    dq = din[:nq].view(B, cfg.h_q, d)
+    dkn = din[nq:nq + nkv].view(B, hkv, d)
+    dvn = din[nq + nkv:].view(B, hkv, d)
+    hout = torch.empty((B, cfg.h_q, d), dtype=torch.float32).pin_memory()
+    dsl = w.seqlens.to(device)
+    ws = torch.zeros(gk.workspace_size(B, cfg.h_q, hkv, d, cfg.n_splits), dtype=torch.uint8, device=device)
+    out = torch.empty((B, cfg.h_q, d), dtype=torch.float32, device=device)
+
+    def step():
+        din.copy_(hin, non_blocking=True)
+        gk.gqa_decode_attn_append(dq, dkn, dvn, kp, vp, dsl, cfg.n_splits, cfg.scale, out=out, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    ms, _ = _timed_region(lambda: [step() for _ in range(E)], device, world)
+    check_status(gk, device, "after the decode-loop end-to-end steps")
+    ms = max_over_ranks(ms / E, world, device)
+    kv = 2 * sum(S + 1 for S in sl) * hkv * d * w.k.element_size()
+    total = sum_over_ranks(float(kv), world, device)
+    del kp, vp, ws
+    return {
+        "value": round(total / (ms * 1e-3) / 1e9, 2),
+        "unit": UNIT,
+        "h2d_bytes_per_step": hin.numel() * hin.element_size(),
+        "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+        "ms_per_step": round(ms, 5),
+        "kv_bytes_per_step": kv,
+        "note": "decode-loop form: the cache resident on the GPU (padded, S_max + 1 rows); q and the new "
+                "token's k, v copied in from one pinned buffer, gqa_decode_attn_append (append + attend over "
+                "S_b + 1 keys), the result copied back; direct calls, every step",
+    }
+
+
 def timed_steps(call, K: int, W: int, device, world: int, graph: bool = True):
     """W untimed warm-up steps, then exactly K steps timed twice: as K direct
     calls of the public API, and (graph=True) as one replay of a CUDA graph of
@@ -545,6 +605,7 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hsl))
     d2h = hout.numel() * hout.element_size()
     e2e_bytes = sum_over_ranks(float(kv_bytes), world, device)
+    loop = decode_loop_e2e(gk, cfg, w, rig, E, device, world) if not cfg.chunk_len else None
     launches = rig.launches
     kernel = rig.kernel_name()
     del rig, dq, dk, dv, dsl
@@ -630,11 +691,13 @@ def run_ours(args, rank, world, local_rank):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
             "ms_per_step": round(e2e_ms, 4),
-            "note": "pinned host q/k/v/seqlens copied in and out copied back every step",
+            "note": "pinned host q/k/v/seqlens (the whole cache) copied in and out copied back every step",
         },
         "gpu_launches": K * launches,
         "clocks": clocks,
     }
+    if loop is not None:
+        line["e2e_decode_loop"] = loop
     if per_config is not None:
         line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:

@@ -57,6 +57,9 @@ def test_decode_bench_line():
     # work only, so the two agree closely
     dc = d["direct_calls"]
     assert 0.5 < dc["ms_per_step"] / d["ms_per_step"] < 2.0
+    # the decode-loop form: only q and the new token move per step
+    lp = d["e2e_decode_loop"]
+    assert 0 < lp["value"] <= 1.2 * d["value"] and lp["h2d_bytes_per_step"] < 1 << 20
     # every other workload, timed the same way
     assert sorted(d["per_config"]) == sorted(n for n in workloads.CONFIGS if n != "llama70b")
     for name, e in d["per_config"].items():
