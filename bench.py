@@ -517,9 +517,10 @@ def per_config_entry(gk, name, args, device, sampler, peak):
         "sha256_q_k_v_seqlens": input_hashes(w),
         "clocks": sampler.summary(win),
     }
+    out = rig.out.detach().cpu()   # the output of the last timed step
     del rig, w
     torch.cuda.empty_cache()
-    return entry
+    return entry, out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -543,6 +544,7 @@ def run_ours(args, rank, world, local_rank):
                                            graph=not args.no_graph)
     total_ms = graph_ms if graph_ms is not None else direct_ms
     check_status(gk, device, "after the timed region")
+    out_host = rig.out.detach().cpu()   # the output of the last timed step
     clocks = sampler.summary(win) if rank == 0 else None
     max_direct_ms = max_over_ranks(direct_ms, world, device)
 
@@ -613,11 +615,12 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_src = measured_hbm_peak()
     per_config = None
+    gpu_outs = {cfg.name: out_host}
     if world == 1 and not args.no_per_config and cfg == workloads.CONFIGS.get(cfg.name):
         per_config = {}
         for name in workloads.CONFIGS:
             if name != cfg.name:
-                per_config[name] = per_config_entry(gk, name, args, device, sampler, peak)
+                per_config[name], gpu_outs[name] = per_config_entry(gk, name, args, device, sampler, peak)
     sampler.stop()
 
     if rank != 0:
@@ -701,8 +704,8 @@ def run_ours(args, rank, world, local_rank):
     if per_config is not None:
         line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
-        line["cpu_baseline"]["single_core"] = single_core_baselines(args.seed)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=20.0, gpu_out=out_host)
+        line["cpu_baseline"]["single_core"] = single_core_baselines(args.seed, gpu_outs=gpu_outs)
     return line
 
 
@@ -716,16 +719,35 @@ def oracle_sample(w, n_items: int, start: int):
     return [(i // c.h_q, i % c.h_q) for i in idx]
 
 
-def cpu_baseline(w, budget_s: float):
+def sample_parity(cfg, items, ref, gpu_out) -> dict:
+    """The GPU output of the timed steps against the oracle rows computed for
+    the CPU baseline: max abs error, max rel error over |ref| >= 0.2, and the
+    worst error as a fraction of the elementwise bound atol + rtol |ref|."""
+    atol, rtol = (2e-3, 1e-2) if cfg.dtype == "bf16" else (1e-5, 1e-5)
+    got = np.stack([gpu_out[b, h].double().numpy() for b, h in items])
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= 0.2
+    worst = float((err / (atol + rtol * np.abs(ref))).max())
+    return {"rows": len(items), "max_abs_err": float(err.max()),
+            "max_rel_err": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+            "worst_err_over_bound": round(worst, 5), "bound": f"{atol:g} + {rtol:g}*|ref|",
+            "pass": bool(worst <= 1.0)}
+
+
+def cpu_baseline(w, budget_s: float, gpu_out=None):
     """Times the oracle as it stands on a sample of (b, h) rows; KV GB/s is
-    the workload's KV bytes scaled by the sampled fraction of its rows."""
+    the workload's KV bytes scaled by the sampled fraction of its rows.  The
+    rows of the first pass also check the GPU output of the timed steps
+    (`gpu_out`, host copy) when it is given."""
     import oracle
     c = w.cfg
     total = c.B * c.h_q
     cores = os.cpu_count() or 1
     n = min(total, max(cores, 1))
     t0 = time.perf_counter()
-    oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=oracle_sample(w, n, 0))
+    first = oracle_sample(w, n, 0)
+    ref0 = oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=first)
     dt = time.perf_counter() - t0
     per_item = dt / n
     n_run = int(max(n, budget_s / max(per_item, 1e-9)))
@@ -738,17 +760,21 @@ def cpu_baseline(w, budget_s: float):
         done += m
     dt = time.perf_counter() - t0
     kv_equiv = w.kv_bytes * done / total
-    return {"value": round(kv_equiv / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{done} (b, h) output rows, cycling through the workload's {total} "
-                      f"({done / total:.2f} passes; fp64 two-pass, {dt:.1f} s); KV bytes "
-                      f"scaled by the rows done",
-            "seconds": round(dt, 2)}
+    res = {"value": round(kv_equiv / dt / 1e9, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"{done} (b, h) output rows, cycling through the workload's {total} "
+                     f"({done / total:.2f} passes; fp64 two-pass, {dt:.1f} s); KV bytes "
+                     f"scaled by the rows done",
+           "seconds": round(dt, 2)}
+    if gpu_out is not None:
+        res["parity"] = sample_parity(c, first, ref0, gpu_out)
+    return res
 
 
-def single_core_baselines(seed, budget_s: float = 2.0) -> dict:
+def single_core_baselines(seed, budget_s: float = 2.0, gpu_outs=None) -> dict:
     """The oracle on ONE host thread for the tiny, Llama-2-7B and Llama-70B
     workloads: (b, h) rows for about `budget_s` each, KV GB/s scaled by the
-    rows done."""
+    rows done.  Rows computed here also check the GPU output of that
+    workload's timed steps when `gpu_outs` holds it."""
     import oracle
     res = {}
     for name in ("tiny", "llama7b", "llama70b"):
@@ -756,15 +782,21 @@ def single_core_baselines(seed, budget_s: float = 2.0) -> dict:
         c = w.cfg
         total = c.B * c.h_q
         done, start, dt = 0, 0, 0.0
+        items, refs = [], []
         while dt < budget_s and done < 64 * total:
+            it = oracle_sample(w, 1, start)
             t0 = time.perf_counter()
-            oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale,
-                        items=oracle_sample(w, 1, start), nthreads=1)
+            r = oracle.attn(w.q, w.k, w.v, w.seqlens, c.h_q, c.h_kv, c.scale, items=it, nthreads=1)
             dt += time.perf_counter() - t0
+            if done < total:
+                items += it
+                refs.append(r[0])
             start += 1
             done += 1
         res[name] = {"value": round(w.kv_bytes * done / total / dt / 1e9, 4), "unit": UNIT, "cores": 1,
                      "sample": f"{done} of {total} (b, h) rows, {dt:.2f} s"}
+        if gpu_outs and name in gpu_outs:
+            res[name]["parity"] = sample_parity(c, items, np.stack(refs), gpu_outs[name])
     return res
 
 
