@@ -657,7 +657,7 @@ int prefill(const void* q, const void* k, const void* v, const int32_t* seqlens,
 
 extern "C" {
 
-int gqa_decode_version(void) { return 100; }
+int gqa_decode_version(void) { return 200; }
 
 const char* gqa_decode_error_string(int status) {
   switch (status) {

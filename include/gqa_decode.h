@@ -85,7 +85,8 @@ typedef enum {
 
 typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
 
-/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+/* Version of this ABI (major * 10000 + minor * 100 + patch): 200 (0.2.0)
+ * adds gqa_decode_fused_plan. */
 GQA_API int gqa_decode_version(void);
 
 /* Human-readable name of a gqa_status value (static storage). */
