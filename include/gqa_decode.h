@@ -103,10 +103,13 @@ GQA_API size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d
                                          int chunk_len, int max_seqlen);
 
 /*
- * Fused decode attention, split by count: one kernel computes every split's
- * triplet and the last split to finish for a (b, kv head) merges them in
- * split order and writes out[b][h][:] for the group's query heads.  The
- * result is identical to gqa_decode_partial followed by mlo_merge.
+ * Fused decode attention, split by count: every split's triplet is computed
+ * and the splits of each (b, kv head) are merged in split order into
+ * out[b][h][:] for the group's query heads -- by the CTA that finishes the
+ * group's last split, or by a second kernel over all rows (see
+ * gqa_decode_fused_plan and gqa_decode_launches_per_call).  The result equals
+ * gqa_decode_partial followed by mlo_merge up to fp32 rounding (bit for bit
+ * on the fp32 path, which shares the per-split kernel).
  *
  * workspace: NULL, or caller device memory of at least
  *   gqa_decode_workspace_size(...) bytes, 256-byte aligned, whose first
