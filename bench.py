@@ -471,7 +471,9 @@ def timed_steps(call, K: int, W: int, device, world: int, graph: bool = True):
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(device)
     side.wait_stream(stream)
-    with torch.cuda.graph(g, stream=side):
+    # thread-local capture: CUDA calls of other host threads (a process
+    # group's watchdog) neither join nor break the capture
+    with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
         for i in range(K):
             call(W + i)
     stream.wait_stream(side)
