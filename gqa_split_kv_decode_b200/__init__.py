@@ -56,18 +56,20 @@ _version = _sig("gqa_decode_version", _ci)
 _errstr = _sig("gqa_decode_error_string", ctypes.c_char_p, _ci)
 _ws_size = _sig("gqa_decode_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci)
 _ws_size_chunked = _sig("gqa_decode_chunked_workspace_size", _sz, _ci, _ci, _ci, _ci, _ci, _ci)
-_attn = _sig("gqa_decode_attn", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _ci,
-             _vp, _sz, _vp)
-_attn_noalloc = _sig("gqa_decode_attn_noalloc", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
-                     _ci, _cf, _ci, _vp)
+_ll = ctypes.c_longlong
+# packed-cache calls: (q, k_cache, v_cache, seqlens, kv_rows, ...)
+_attn = _sig("gqa_decode_attn", _ci, _vp, _vp, _vp, _vp, _ll, _vp, _ci, _ci, _ci, _ci, _ci, _cf,
+             _ci, _vp, _sz, _vp)
+_attn_noalloc = _sig("gqa_decode_attn_noalloc", _ci, _vp, _vp, _vp, _vp, _ll, _vp, _ci, _ci, _ci,
+                     _ci, _ci, _cf, _ci, _vp)
 _attn_append = _sig("gqa_decode_attn_append", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci,
                     _ci, _ci, _ci, _ci, _cf, _ci, _vp, _sz, _vp)
-_attn_chunked = _sig("gqa_decode_attn_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
-                     _ci, _ci, _cf, _ci, _vp, _sz, _vp)
-_partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
-                _ci, _cf, _ci, _vp)
-_partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _ci,
-                        _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
+_attn_chunked = _sig("gqa_decode_attn_chunked", _ci, _vp, _vp, _vp, _vp, _ll, _vp, _ci, _ci, _ci,
+                     _ci, _ci, _ci, _cf, _ci, _vp, _sz, _vp)
+_partial = _sig("gqa_decode_partial", _ci, _vp, _vp, _vp, _vp, _ll, _vp, _vp, _vp, _ci, _ci, _ci,
+                _ci, _ci, _cf, _ci, _vp)
+_partial_chunked = _sig("gqa_decode_partial_chunked", _ci, _vp, _vp, _vp, _vp, _ll, _vp, _vp, _vp,
+                        _ci, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp)
 _merge = _sig("mlo_merge", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _vp)
 _merge_ranked = _sig("mlo_merge_ranked", _ci, _vp, _vp, _vp, _vp, _ci, _ci, _ci, _ci,
                      ctypes.c_longlong, ctypes.c_longlong, _vp)
@@ -239,7 +241,7 @@ def gqa_decode_attn(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, out
     out = _out_idx(out, (B, h_q, d), idx)
     wp, wb = _ws(workspace, idx, _ws_size, B, h_q, h_kv, d, n_splits)
     _check(_on(idx, _attn, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-               out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt, wp, wb,
+               k_cache.shape[0], out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt, wp, wb,
                _stream(idx)), "gqa_decode_attn")
     return out
 
@@ -256,7 +258,7 @@ def gqa_decode_attn_noalloc(q, k_cache, v_cache, seqlens, n_splits: int, scale=N
     B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
     out = _out_idx(out, (B, h_q, d), idx)
     _check(_on(idx, _attn_noalloc, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-               out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
+               k_cache.shape[0], out.data_ptr(), B, h_q, h_kv, d, n_splits, _default_scale(d, scale), dt,
                _stream(idx)), "gqa_decode_attn_noalloc")
     return out
 
@@ -291,7 +293,7 @@ def gqa_decode_attn_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max_se
     out = _out_idx(out, (B, h_q, d), idx)
     wp, wb = _ws(workspace, idx, _ws_size_chunked, B, h_q, h_kv, d, chunk_len, max_seqlen)
     _check(_on(idx, _attn_chunked, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-               out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
+               k_cache.shape[0], out.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen, _default_scale(d, scale), dt,
                wp, wb, _stream(idx)), "gqa_decode_attn_chunked")
     return out
 
@@ -308,7 +310,7 @@ def gqa_decode_partial(q, k_cache, v_cache, seqlens, n_splits: int, scale=None, 
     B, h_q, h_kv, d, dt, idx = _inputs(q, k_cache, v_cache, seqlens)
     m, l, o = _triplets(B, h_q, n_splits, d, idx, m, l, o)
     _check(_on(idx, _partial, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-               m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
+               k_cache.shape[0], m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, n_splits,
                _default_scale(d, scale), dt, _stream(idx)), "gqa_decode_partial")
     return m, l, o
 
@@ -320,7 +322,7 @@ def gqa_decode_partial_chunked(q, k_cache, v_cache, seqlens, chunk_len: int, max
     n = max(1, -(-max_seqlen // chunk_len)) if chunk_len > 0 and max_seqlen >= 0 else 1
     m, l, o = _triplets(B, h_q, n, d, idx, m, l, o)
     _check(_on(idx, _partial_chunked, q.data_ptr(), _ptr(k_cache), _ptr(v_cache), seqlens.data_ptr(),
-               m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
+               k_cache.shape[0], m.data_ptr(), l.data_ptr(), o.data_ptr(), B, h_q, h_kv, d, chunk_len, max_seqlen,
                _default_scale(d, scale), dt, _stream(idx)), "gqa_decode_partial_chunked")
     return m, l, o
 

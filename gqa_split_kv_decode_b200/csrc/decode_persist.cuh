@@ -58,13 +58,14 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 // u < that number -- unit u itself.  A unit is a non-empty split of one
 // (b, kv head / head block); units are numbered b-major, then kv head / head
 // block, then split.
+template <bool HINT = false>
 __device__ Unit scan_units(const DecodeArgs& a, int H, int u, int lane, int* total) {
   int units = 0, rows = 0;
   Unit x{};
   bool found = false;
   for (int base = 0; base < a.B; base += 32) {
     const int b = base + lane;
-    const SeqKeys kk = seq_keys(a, b < a.B ? __ldg(a.seqlens + b) : 0);
+    const SeqKeys kk = seq_keys(a, b < a.B ? load_seqlen<HINT>(a.seqlens + b) : 0);
     int L;
     const int n = b < a.B ? active_splits(a, kk.total, L) : 0;
     const int cu = H * n, cr = kk.cached;
@@ -199,17 +200,40 @@ __global__ void __launch_bounds__(NW * 32)
     for (int i = 0; i < NW * NS; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
     fence_barrier_init();
   }
+  if (a.hint_tiles > 0 && blockIdx.x < a.hint_ctas) {
+    // While the previous grid drains: L2 prefetch of this warp's first tiles
+    // of the CTA's first unit, at rows from lengths read before the wait
+    // (possibly stale, so every box is checked against the cache's rows; the
+    // units are scanned again after the wait).
+    const Unit h = scan_units<true>(a, H, blockIdx.x, lane, nullptr);
+    if (lane == 0)
+      for (int s = 0; s < a.hint_tiles; ++s) {
+        const int t = warp + s * NW;
+        if (t >= h.ntiles) break;
+        const int ts = h.lo + t * kTileKeys;
+        const long long row =
+            h.off + ((ts + kTileKeys <= h.cached_hi) ? ts : h.cached_hi - kTileKeys);
+        if (row >= 0 && row + kTileKeys <= a.kv_rows)
+          tc_prefetch_stage<D>(&kmap, &vmap, h.gy / a.n_hb, (int)row);
+      }
+  }
   grid_dependency_wait();
   allow_dependent_launch();
   __syncthreads();
 
   if (blockIdx.x == 0 && threadIdx.x < 32) {  // report bad lengths once
+    long long rows = 0;
     for (int b = lane; b < a.B; b += 32) {
       const int S = __ldg(a.seqlens + b);
       report_length(a, S, true);
       if (a.chunk_len > 0 && (long long)seq_keys(a, S).total > (long long)a.n_slots * a.chunk_len)
         raise_status(kStatusSeqlenOverMax);
+      rows += S > 0 ? S : 0;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rows += __shfl_xor_sync(kFull, rows, o);
+    if (lane == 0 && a.cap == 0 && a.kv_rows >= 0 && rows > a.kv_rows)  // cache rows past the cache
+      raise_status(kStatusSeqlenOverMax);
   }
 
   int A32 = 0;

@@ -67,9 +67,10 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int j = j0 + u * NW;
-      if (j < sp.hi) {
-        // key j comes from the cache, or is the appended token (key number cached_hi)
-        const bool fresh = sp.has_new && j == sp.cached_hi;
+      // key j comes from the cache, or is the appended token (key number cached_hi);
+      // a cache row past the cache's rows reads as zero
+      const bool fresh = sp.has_new && j == sp.cached_hi;
+      if (j < sp.hi && (fresh || a.kv_rows < 0 || sp.off + j < a.kv_rows)) {
         const size_t base = fresh ? new_base : ((size_t)(sp.off + j) * a.h_kv + g) * D + lane * PER;
         const float* ksrc = fresh ? static_cast<const float*>(a.k_new) : kp;
         const float* vsrc = fresh ? static_cast<const float*>(a.v_new) : vp;

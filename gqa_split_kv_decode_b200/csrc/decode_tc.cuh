@@ -298,6 +298,15 @@ __device__ __forceinline__ void tc_issue_stage(uint32_t dst, uint32_t bar, const
     tma_load_3d(dst + (HALVES + h) * kBoxBytes, vmap, h * 64, g, row, bar, policy);
 }
 
+template <int D>
+__device__ __forceinline__ void tc_prefetch_stage(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                                  int g, int row) {
+#pragma unroll
+  for (int h = 0; h < TcShape<D>::kHalves; ++h) tma_prefetch_3d(kmap, h * 64, g, row);
+#pragma unroll
+  for (int h = 0; h < TcShape<D>::kHalves; ++h) tma_prefetch_3d(vmap, h * 64, g, row);
+}
+
 // 1024-byte-aligned start of the dynamic shared memory (128-byte swizzle
 // atoms repeat every 1024 bytes).
 __device__ __forceinline__ uint8_t* aligned_dyn_smem(uint8_t* p) {
@@ -336,6 +345,21 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
     for (int i = 0; i < NW * NS; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
     fence_barrier_init();
+  }
+  if (a.hint_tiles > 0 &&
+      blockIdx.x + gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z) < a.hint_ctas) {
+    // While the previous grid drains: L2 prefetch of this warp's first tiles,
+    // at rows from lengths read before the wait (possibly stale, so every
+    // box is checked against the cache's rows; the split is located again
+    // after the wait).
+    const Split h = locate_split<true>(a, b, slot, lane, false);
+    if (lane == 0 && slot < h.n_active)
+      for (int s = 0; s < a.hint_tiles; ++s) {
+        const int ts = h.lo + (warp + s * NW) * KT;
+        if (ts >= h.cached_hi) break;
+        const long long row = h.off + ((ts + KT <= h.cached_hi) ? ts : h.cached_hi - KT);
+        if (row >= 0 && row + KT <= a.kv_rows) tc_prefetch_stage<D>(&kmap, &vmap, g, (int)row);
+      }
   }
   grid_dependency_wait();
   allow_dependent_launch();

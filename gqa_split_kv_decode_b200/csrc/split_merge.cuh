@@ -29,6 +29,11 @@ struct DecodeArgs {
   const void* k_new;        // append: the new token's k and v, [B][h_kv][D]; null otherwise
   const void* v_new;
   long long cap;            // > 0: cache rows per sequence ([B][cap][h_kv][D]); 0: packed
+  long long kv_rows;        // rows of the cache; no cache row at or past it is read.  < 0:
+                            //   not given (packed calls that do not pass it)
+  int hint_tiles;           // > 0: a CTA prefetches its warps' first hint_tiles tiles into L2
+                            //   before the dependency wait (needs kv_rows >= 0)
+  int hint_ctas;            // only CTAs whose linear index is below it prefetch (first wave)
   int B, h_q, h_kv, G, n_hb;
   int n_splits;             // > 0: split by count
   int chunk_len;            // > 0: split by fixed chunks
@@ -81,6 +86,14 @@ struct Split {
 // warp).  Split i covers [i*L, min((i+1)*L, S)) with L = ceil(S / n_splits)
 // or L = chunk_len.  n_active = max(1, ceil(S / L)): the number of splits
 // the fused merge waits for (split 0 stands in for an empty sequence).
+// HINT: lengths read with relaxed loads before the dependency wait, for L2
+// prefetch addresses only (the split is located again after the wait).
+template <bool HINT = false>
+__device__ __forceinline__ int load_seqlen(const int32_t* p) {
+  return HINT ? ld_relaxed_s32(p) : __ldg(p);
+}
+
+template <bool HINT = false>
 __device__ __forceinline__ Split locate_split(const DecodeArgs& a, int b, int slot, int lane,
                                               bool report) {
   long long acc = 0;
@@ -88,14 +101,17 @@ __device__ __forceinline__ Split locate_split(const DecodeArgs& a, int b, int sl
     acc = (long long)b * a.cap;
   } else {
     for (int j = lane; j < b; j += 32) {
-      const int s = __ldg(a.seqlens + j);
+      const int s = load_seqlen<HINT>(a.seqlens + j);
       acc += s > 0 ? s : 0;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
   }
-  const int Sraw = __ldg(a.seqlens + b);
+  const int Sraw = load_seqlen<HINT>(a.seqlens + b);
   report_length(a, Sraw, report);
+  // the sequence's cache rows end past the cache
+  if (report && a.cap == 0 && a.kv_rows >= 0 && acc + (Sraw > 0 ? Sraw : 0) > a.kv_rows)
+    raise_status(kStatusSeqlenOverMax);
   const SeqKeys kk = seq_keys(a, Sraw);
   const int S = kk.total;
   const long long L =

@@ -22,6 +22,7 @@
  *   k_cache  [sum_b S_b][h_kv][d_head]   dtype, packed: sequence b occupies
  *   v_cache  [sum_b S_b][h_kv][d_head]   rows S_0 + ... + S_{b-1} onwards
  *   seqlens  int32 [B]                   S_b (device memory)
+ *   kv_rows  rows of k_cache and v_cache (host value), or -1 if not known
  *   out      fp32 [B][h_q][d_head]       O = o / l (0 where S_b == 0)
  *   m, l     fp32 [B][h_q][n_slots]      per-split triplets (m in natural
  *   o        fp32 [B][h_q][n_slots][d_head]   log units, o unnormalised)
@@ -55,6 +56,17 @@
  *   (rows [0, sum_b S_b)); rows of a neighbouring sequence that fall inside a
  *   loaded tile are masked by index, so they must hold finite values (any
  *   packed cache does).
+ * - kv_rows (packed-cache calls): the number of rows the caller allocated
+ *   for k_cache and v_cache (each is [kv_rows][h_kv][d_head]).  When it is
+ *   given (>= 1), no cache row at or past it is read: rows past it read as
+ *   zero, and sum_b S_b > kv_rows sets GQA_ERR_DEVICE_SEQLEN in the status
+ *   word.  kv_rows = 0 is an empty cache (every S_b must be 0).  Knowing it
+ *   also lets the bf16 kernels issue L2 prefetches of their first K/V tiles
+ *   before the kernel that precedes them on the stream has finished (the
+ *   lengths they read for that may not be final yet; every prefetched row is
+ *   checked against kv_rows, and the result never depends on it).
+ *   kv_rows = -1: not known -- no clipping, no early prefetch; values below
+ *   -1 are GQA_ERR_INVALID_ARG, values above 2^31 - 1 GQA_ERR_UNSUPPORTED.
  */
 #ifndef GQA_DECODE_H
 #define GQA_DECODE_H
@@ -85,8 +97,9 @@ typedef enum {
 
 typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
 
-/* Version of this ABI (major * 10000 + minor * 100 + patch): 200 (0.2.0)
- * adds gqa_decode_fused_plan. */
+/* Version of this ABI (major * 10000 + minor * 100 + patch): 300 (0.3.0)
+ * adds the kv_rows argument of the packed-cache calls; 0.2.0 added
+ * gqa_decode_fused_plan. */
 GQA_API int gqa_decode_version(void);
 
 /* Human-readable name of a gqa_status value (static storage). */
@@ -123,7 +136,7 @@ GQA_API size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d
  *   device); calls that use it must be ordered on one stream.
  */
 GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_cache,
-                    const int32_t *seqlens, float *out,
+                    const int32_t *seqlens, long long kv_rows, float *out,
                     int B, int h_q, int h_kv, int d_head, int n_splits, float scale,
                     int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
@@ -151,7 +164,7 @@ GQA_API int gqa_decode_attn(const void *q, const void *k_cache, const void *v_ca
  * them on one stream.
  */
 GQA_API int gqa_decode_attn_noalloc(const void *q, const void *k_cache, const void *v_cache,
-                                    const int32_t *seqlens, float *out,
+                                    const int32_t *seqlens, long long kv_rows, float *out,
                                     int B, int h_q, int h_kv, int d_head, int n_splits,
                                     float scale, int dtype, void *stream);
 
@@ -171,7 +184,9 @@ GQA_API int gqa_decode_attn_noalloc(const void *q, const void *k_cache, const vo
  * workspace and the result are as for gqa_decode_attn.  Only the new rows
  * are written; no other cache row is read or written outside [0, S_b + 1)
  * of each sequence, except that rows of the previous sequence's unused tail
- * may be read into a masked, zeroed tile.
+ * may be read into a masked, zeroed tile.  The cache's B * cache_capacity
+ * rows play the part of kv_rows (the early L2 prefetch of the bf16 kernels
+ * stays inside them).
  */
 GQA_API int gqa_decode_attn_append(const void *q, const void *k_new, const void *v_new,
                                    void *k_cache, void *v_cache, const int32_t *seqlens,
@@ -187,7 +202,7 @@ GQA_API int gqa_decode_attn_append(const void *q, const void *k_new, const void 
  * the status word and only its first n_slots chunks are used.
  */
 GQA_API int gqa_decode_attn_chunked(const void *q, const void *k_cache, const void *v_cache,
-                            const int32_t *seqlens, float *out,
+                            const int32_t *seqlens, long long kv_rows, float *out,
                             int B, int h_q, int h_kv, int d_head, int chunk_len, int max_seqlen,
                             float scale, int dtype, void *workspace, size_t workspace_bytes,
                             void *stream);
@@ -199,14 +214,15 @@ GQA_API int gqa_decode_attn_chunked(const void *q, const void *k_cache, const vo
  * natural-log units, o unnormalised, empty split = (-inf, 0, 0)).
  */
 GQA_API int gqa_decode_partial(const void *q, const void *k_cache, const void *v_cache,
-                       const int32_t *seqlens, float *m, float *l, float *o,
+                       const int32_t *seqlens, long long kv_rows, float *m, float *l, float *o,
                        int B, int h_q, int h_kv, int d_head, int n_splits, float scale,
                        int dtype, void *stream);
 
 /* Partial attention with the chunked split policy (n_slots triplets per row,
  * n_slots = max(1, ceil(max_seqlen / chunk_len))). */
 GQA_API int gqa_decode_partial_chunked(const void *q, const void *k_cache, const void *v_cache,
-                               const int32_t *seqlens, float *m, float *l, float *o,
+                               const int32_t *seqlens, long long kv_rows, float *m, float *l,
+                               float *o,
                                int B, int h_q, int h_kv, int d_head, int chunk_len,
                                int max_seqlen, float scale, int dtype, void *stream);
 

@@ -28,9 +28,11 @@ def lib():
     path = _builder().build()
     lib = ctypes.CDLL(path)
     vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    lib.gqa_decode_attn.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
-    lib.gqa_decode_attn_chunked.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
-    lib.gqa_decode_partial.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
+    ll = ctypes.c_longlong
+    lib.gqa_decode_attn.argtypes = [vp, vp, vp, vp, ll, vp, ci, ci, ci, ci, ci, cf, ci, vp, sz, vp]
+    lib.gqa_decode_attn_chunked.argtypes = [vp, vp, vp, vp, ll, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp, sz,
+                                            vp]
+    lib.gqa_decode_partial.argtypes = [vp, vp, vp, vp, ll, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp]
     lib.mlo_merge.argtypes = [vp, vp, vp, vp, ci, ci, ci, vp]
     lib.gqa_prefill_attn.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
     lib.gqa_decode_workspace_size.restype = sz
@@ -104,18 +106,22 @@ FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation
     (dict(ws=FAKE, ws_bytes=16), WORKSPACE),  # caller workspace too small
     (dict(ws=FAKE + 16, ws_bytes=1 << 30), WORKSPACE),  # not 256-byte aligned
     (dict(B=0), OK),                         # empty batch: nothing to do
+    (dict(B=0, kv_rows=-1), OK),             # cache rows not given
+    (dict(kv_rows=-2), INVALID),             # below -1
+    (dict(kv_rows=1 << 31), UNSUPPORTED),    # past int32 row coordinates
 ])
 def test_fused_argument_checks(lib, kw, expect):
-    a = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, out=FAKE, B=1, h_q=8, h_kv=2, d=128, n_splits=4,
-             scale=0.1, dtype=1, ws=None, ws_bytes=0)
+    a = dict(q=FAKE, k=FAKE, v=FAKE, sl=FAKE, kv_rows=100, out=FAKE, B=1, h_q=8, h_kv=2, d=128,
+             n_splits=4, scale=0.1, dtype=1, ws=None, ws_bytes=0)
     a.update(kw)
-    rc = lib.gqa_decode_attn(a["q"], a["k"], a["v"], a["sl"], a["out"], a["B"], a["h_q"], a["h_kv"],
-                             a["d"], a["n_splits"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"], None)
+    rc = lib.gqa_decode_attn(a["q"], a["k"], a["v"], a["sl"], a["kv_rows"], a["out"], a["B"], a["h_q"],
+                             a["h_kv"], a["d"], a["n_splits"], a["scale"], a["dtype"], a["ws"],
+                             a["ws_bytes"], None)
     assert rc == expect
 
 
 def test_chunked_argument_checks(lib):
-    args = [FAKE] * 5
+    args = [FAKE] * 4 + [100, FAKE]   # q, k, v, seqlens, kv_rows, out
     assert lib.gqa_decode_attn_chunked(*args, 1, 8, 2, 128, 0, 100, 0.1, 1, None, 0, None) == INVALID
     assert lib.gqa_decode_attn_chunked(*args, 1, 8, 2, 128, 16, -1, 0.1, 1, None, 0, None) == INVALID
     # 1025 chunks of 1 key exceeds the 1024 triplet slots
@@ -123,7 +129,7 @@ def test_chunked_argument_checks(lib):
 
 
 def test_partial_and_merge_argument_checks(lib):
-    p_null = [FAKE] * 4 + [0, FAKE, FAKE]
+    p_null = [FAKE] * 4 + [100, 0, FAKE, FAKE]   # q, k, v, seqlens, kv_rows, m = NULL, l, o
     assert lib.gqa_decode_partial(*p_null, 1, 8, 2, 128, 4, 0.1, 1, None) == INVALID
     assert lib.mlo_merge(FAKE, FAKE, FAKE, FAKE, 0, 4, 128, None) == OK     # no rows: no launch
     assert lib.mlo_merge(FAKE, FAKE, FAKE, FAKE, 4, 0, 128, None) == INVALID
