@@ -180,9 +180,11 @@ constexpr int kTcStages = GQA_TC_STAGES;
 
 // Tiles per warp that the bf16 kernels' first-wave CTAs prefetch into L2
 // before their dependency wait (-DGQA_HINT_TILES overrides it; 0: none).
-// Measured on B200 over back-to-back calls: 3 and 6 tiles took the 70B-shaped
-// call from 47.8 to 46.3 and 45.9 us and the 7B-shaped one from 16.6 to 15.6
-// and 15.1 us.
+// Measured on B200 over 2000 back-to-back calls: none, 6, 8 and 12 tiles ran
+// the 70B-shaped call (B 8, 64/8 heads, 8192 keys) in 46.7, 45.6, 46.0 and
+// 46.7 us and the 7B-shaped one (B 1, 32/32 heads, 4096 keys) in 16.6, 14.8,
+// 15.3 and 15.3 us; deeper prefetches evict each other and delay the
+// running call's own loads.
 #ifndef GQA_HINT_TILES
 #define GQA_HINT_TILES 6
 #endif
