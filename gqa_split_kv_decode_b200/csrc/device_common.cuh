@@ -196,6 +196,13 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, 
                : "memory");
 }
 
+// atomicAdd with gpu-scope acquire-release semantics; returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // A gpu-scope relaxed load: may run concurrently with another grid's store
 // to the same word (it returns the old or the new value) and is not served
 // from the SM's incoherent caches.

@@ -308,25 +308,31 @@ __device__ __forceinline__ void merge_row_warp(const float* m, const float* l, c
 // group's rows over the n_active splits and writes `out`.  Nothing waits on
 // another CTA, so there is no inter-CTA spin.  The last CTA also resets the
 // ticket to 0 for the next call.
+//
+// Ordering: the barrier puts every thread's triplet stores before thread 0's
+// ticket; the ticket is a gpu-scope acq_rel atomic, so it releases them
+// (cumulatively) to the CTA that takes the last ticket, and that CTA's
+// acquire, passed on to its other threads by the second barrier, makes every
+// released triplet visible to the merge's L2 loads.  The reset needs no
+// ordering within the call: no CTA of this call takes the ticket after the
+// last one, and the next call reads it only after this grid has ended.
 template <int NW, int HB, int D>
 __device__ void fused_finish(const DecodeArgs& a, int b, int g, int hb, int n_active,
                              int* sm_flag) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
     const long long ti = (long long)b * gridDim.y + blockIdx.y;
     int last = 0;
     if (in_bounds(ti, kTicketCount, kSiteTicket)) {
       int* t = a.tickets + ti;
-      const int prev = atomicAdd(t, 1);
+      const int prev = atom_add_acq_rel_gpu(t, 1);
       last = (prev == n_active - 1);
-      if (last) atomicExch(t, 0);
+      if (last) *t = 0;
     }
     *sm_flag = last;
   }
   __syncthreads();
   if (!*sm_flag) return;
-  __threadfence();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int hh = warp; hh < HB; hh += NW) {
     const int gi = hb * HB + hh;
