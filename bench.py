@@ -73,6 +73,9 @@ def parse_args(argv=None):
     p.add_argument("--batch", type=int, default=None, help="decode: override the workload's B")
     p.add_argument("--no-graph", action="store_true",
                    help="time the K steps as direct calls only (no CUDA-graph replay)")
+    p.add_argument("--no-hold", action="store_true",
+                   help="start the timed region on an idle GPU (no device-side hold before the "
+                        "start event), so the host's first submission falls inside it")
     p.add_argument("--no-per-config", action="store_true",
                    help="decode: time only the headline workload (skip the per_config object)")
     p.add_argument("--seed", type=int, default=None,
@@ -373,10 +376,21 @@ def upload_graph(g, stream) -> bool:
         return False
 
 
-def _timed_region(run, device, world):
+# Device cycles of the stream hold queued before a device-timed region
+# (about 0.1 ms at the B200's clocks).
+HOLD_CYCLES = 200_000
+
+
+def _timed_region(run, device, world, hold: bool = False):
     """One timed region: barrier + synchronize, CUDA events on the launching
     stream around run(), synchronize + barrier.  Returns (device ms, host
-    wall window)."""
+    wall window).
+
+    hold: queue a bounded spin (torch.cuda._sleep, HOLD_CYCLES) ahead of the
+    start event, so the GPU is still busy with it while the host submits
+    run()'s work; the region then starts when the first step does, not when
+    the host's submission reaches an idle GPU (the blocking-kernel method of
+    GPU benchmark harnesses).  Every step of run() stays inside the region."""
     stream = torch.cuda.current_stream(device)
     if world > 1:
         import torch.distributed as dist
@@ -384,6 +398,9 @@ def _timed_region(run, device, world):
     torch.cuda.synchronize(device)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.time()
+    if hold:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(HOLD_CYCLES)
     s.record(stream)
     run()
     e.record(stream)
@@ -454,18 +471,18 @@ def decode_loop_e2e(gk, cfg, w, rig, E: int, device, world: int):
     }
 
 
-def timed_steps(call, K: int, W: int, device, world: int, graph: bool = True):
+def timed_steps(call, K: int, W: int, device, world: int, graph: bool = True, hold: bool = True):
     """W untimed warm-up steps, then exactly K steps timed twice: as K direct
     calls of the public API, and (graph=True) as one replay of a CUDA graph of
     those same K calls, captured and uploaded before its timed region -- every
     step's kernels run unchanged; only the host's launch work leaves the
-    timed region.  Returns (direct ms, graph ms or None, the graph's host
-    window or the direct one)."""
+    timed region.  hold: see _timed_region.  Returns (direct ms, graph ms or
+    None, the graph's host window or the direct one)."""
     stream = torch.cuda.current_stream(device)
     for i in range(W):
         call(i)
     torch.cuda.synchronize(device)
-    direct_ms, win = _timed_region(lambda: [call(W + i) for i in range(K)], device, world)
+    direct_ms, win = _timed_region(lambda: [call(W + i) for i in range(K)], device, world, hold)
     if not graph:
         return direct_ms, None, win
     g = torch.cuda.CUDAGraph()
@@ -479,7 +496,7 @@ def timed_steps(call, K: int, W: int, device, world: int, graph: bool = True):
     stream.wait_stream(side)
     upload_graph(g, stream)
     torch.cuda.synchronize(device)
-    graph_ms, win = _timed_region(g.replay, device, world)
+    graph_ms, win = _timed_region(g.replay, device, world, hold)
     del g
     return direct_ms, graph_ms, win
 
@@ -497,7 +514,7 @@ def per_config_entry(gk, name, args, device, sampler, peak):
     w = workloads.generate(cfg, seed=args.seed)
     rig = DecodeRig(gk, cfg, w, device)
     direct_ms, graph_ms, win = timed_steps(rig.fused, args.steps, args.warmup, device, 1,
-                                           graph=not args.no_graph)
+                                           graph=not args.no_graph, hold=not args.no_hold)
     check_status(gk, device, f"after timing {name}")
     us = (graph_ms if graph_ms is not None else direct_ms) * 1e3 / args.steps
     us_direct = direct_ms * 1e3 / args.steps
@@ -507,7 +524,8 @@ def per_config_entry(gk, name, args, device, sampler, peak):
         "us_per_call": round(us, 3),
         "value_gbs": round(gbs, 2),
         "frac_of_hbm_peak": round(gbs / peak, 4),
-        "timing": "CUDA graph of the K calls" if graph_ms is not None else "direct calls",
+        "timing": ("CUDA graph of the K calls" if graph_ms is not None else "direct calls")
+                  + ("" if args.no_hold else ", device spin queued ahead of the start event"),
         "direct_calls_us_per_call": round(us_direct, 3),
         "direct_calls_frac_of_hbm_peak": round(rig.kv_bytes / (us_direct * 1e-6) / 1e9 / peak, 4),
         "kv_bytes_per_step": rig.kv_bytes,
@@ -543,7 +561,7 @@ def run_ours(args, rank, world, local_rank):
 
     K = args.steps
     direct_ms, graph_ms, win = timed_steps(rig.fused, K, args.warmup, device, world,
-                                           graph=not args.no_graph)
+                                           graph=not args.no_graph, hold=not args.no_hold)
     total_ms = graph_ms if graph_ms is not None else direct_ms
     check_status(gk, device, "after the timed region")
     out_host = rig.out.detach().cpu()   # the output of the last timed step
@@ -565,7 +583,7 @@ def run_ours(args, rank, world, local_rank):
 
     # the same workload through the two-call form: gqa_decode_partial + mlo_merge
     pm_direct, pm_graph, _ = timed_steps(rig.partial_merge, K, args.warmup, device, world,
-                                         graph=not args.no_graph)
+                                         graph=not args.no_graph, hold=not args.no_hold)
     check_status(gk, device, "after timing partial + merge")
     max_pm_ms = max_over_ranks(pm_graph if pm_graph is not None else pm_direct, world, device)
 
@@ -670,7 +688,10 @@ def run_ours(args, rank, world, local_rank):
                        "launch work out of the timed region); a step's launches together, so the dominant "
                        "kernel's own rate is at least this" if graph_ms is not None else
                        "CUDA events around the K back-to-back calls of the timed region (a step's launches "
-                       "together, so the dominant kernel's own rate is at least this)"),
+                       "together, so the dominant kernel's own rate is at least this)")
+                      + ("; a bounded device spin (torch.cuda._sleep) queued ahead of the start event keeps "
+                         "the GPU busy while the host submits the steps, so the region starts with the first "
+                         "step" if not args.no_hold else "; the region starts on an idle GPU"),
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(max_iso_ms, 6),
             "isolated_launch_ms_p10_p90": [round(iso_p10, 6), round(iso_p90, 6)],
@@ -1029,6 +1050,9 @@ def run_prefill(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(device)
     sampler.mark_begin()
+    if not args.no_hold:  # as in _timed_region
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(HOLD_CYCLES)
     t_start.record(stream)
     for i in range(K):
         call(i)
