@@ -55,7 +55,9 @@
  * - No stray reads: a kernel reads only cache rows that belong to the batch
  *   (rows [0, sum_b S_b)); rows of a neighbouring sequence that fall inside a
  *   loaded tile are masked by index, so they must hold finite values (any
- *   packed cache does).
+ *   packed cache does).  The one exception is the early L2 prefetch (see
+ *   kv_rows): it brings rows into the L2 cache only, never into a result,
+ *   and may touch any row below kv_rows.
  * - kv_rows (packed-cache calls): the number of rows the caller allocated
  *   for k_cache and v_cache (each is [kv_rows][h_kv][d_head]).  When it is
  *   given (>= 1), no cache row at or past it is read: rows past it read as
