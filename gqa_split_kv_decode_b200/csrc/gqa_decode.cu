@@ -183,10 +183,11 @@ constexpr int kTcStages = GQA_TC_STAGES;
 // Measured on B200 over 2000 back-to-back calls: none, 6, 8 and 12 tiles ran
 // the 70B-shaped call (B 8, 64/8 heads, 8192 keys) in 46.7, 45.6, 46.0 and
 // 46.7 us and the 7B-shaped one (B 1, 32/32 heads, 4096 keys) in 16.6, 14.8,
-// 15.3 and 15.3 us; deeper prefetches evict each other and delay the
-// running call's own loads.
+// 15.3 and 15.3 us; on another box 4, 5, 6 and 7 tiles ran them in 45.2,
+// 45.1, 45.1, 45.4 and 14.4, 14.25, 14.5, 14.8 us.  Deeper prefetches evict
+// each other and delay the running call's own loads.
 #ifndef GQA_HINT_TILES
-#define GQA_HINT_TILES 6
+#define GQA_HINT_TILES 5
 #endif
 constexpr int kHintTiles = GQA_HINT_TILES;
 
