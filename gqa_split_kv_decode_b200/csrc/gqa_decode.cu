@@ -191,7 +191,16 @@ constexpr int kTcStages = GQA_TC_STAGES;
 #endif
 constexpr int kHintTiles = GQA_HINT_TILES;
 
-int sm_count();
+int sm_count() {
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return -1;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 // CTAs of `kern` resident on the current device at once (per-device cache).
 template <typename K>
@@ -230,16 +239,6 @@ int launch_tc(DecodeArgs a, dim3 grid, cudaStream_t st) {
   return launch_pdl(kern, grid, dim3(NW * 32), smem, st, kmap, vmap, a);
 }
 
-int sm_count() {
-  static std::atomic<int> cached[kMaxDevices];
-  const int dev = current_device();
-  if (dev < 0 || dev >= kMaxDevices) return -1;
-  int n = cached[dev].load(std::memory_order_relaxed);
-  if (n > 0) return n;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-  cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
 
 // Launch plans of the fused bf16 path, chosen from the grid size alone (the
 // sequence lengths live on the device).  R = CTAs of the per-split kernel
@@ -733,9 +732,8 @@ size_t gqa_decode_chunked_workspace_size(int B, int h_q, int h_kv, int d_head, i
 
 int gqa_decode_attn(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* seqlens, long long kv_rows, float* out, int B, int h_q,
-                    int h_kv, int d_head,
-                    int n_splits, float scale, int dtype, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+                    int h_kv, int d_head, int n_splits, float scale, int dtype, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   if (n_splits == 0 && B > 0) {
     n_splits = auto_splits(B, h_q, h_kv, d_head, 0);
     if (n_splits < 0) return -n_splits;
