@@ -4,7 +4,9 @@
 // The per-split grid runs one CTA per (split, kv head, head block, b); when
 // there are more splits than resident CTAs the second wave starts cold and
 // every wave pays its start-up and drain with the memory system idle.  Here
-// the grid is exactly the CTAs that fit at once, and CTA c takes the
+// the grid is C CTAs that all fit at once -- as few as take the units in the
+// same number of rounds, so every CTA gets the same number of units (to
+// one) -- and CTA c takes the
 // non-empty splits ("units") c, c + C, c + 2C, ... in the per-split grid's
 // order (split fastest, then kv head / head block, then b), so CTAs that run
 // together still read neighbouring cache rows.  Each warp keeps one TMA ring
