@@ -377,8 +377,20 @@ def upload_graph(g, stream) -> bool:
 
 
 # Device cycles of the stream hold queued before a device-timed region
-# (about 0.1 ms at the B200's clocks).
+# (about 0.1 ms at the B200's clocks).  torch.cuda._sleep is torch's own
+# bounded spin kernel (a private helper): without it the regions start on an
+# idle GPU, and the JSON line says so.
 HOLD_CYCLES = 200_000
+HOLD_AVAILABLE = hasattr(torch.cuda, "_sleep")
+
+
+def hold_stream(stream):
+    """Queues the bounded spin on `stream`; False when torch lacks it."""
+    if not HOLD_AVAILABLE:
+        return False
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(HOLD_CYCLES)
+    return True
 
 
 def _timed_region(run, device, world, hold: bool = False):
@@ -399,8 +411,7 @@ def _timed_region(run, device, world, hold: bool = False):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.time()
     if hold:
-        with torch.cuda.stream(stream):
-            torch.cuda._sleep(HOLD_CYCLES)
+        hold_stream(stream)
     s.record(stream)
     run()
     e.record(stream)
@@ -525,7 +536,7 @@ def per_config_entry(gk, name, args, device, sampler, peak):
         "value_gbs": round(gbs, 2),
         "frac_of_hbm_peak": round(gbs / peak, 4),
         "timing": ("CUDA graph of the K calls" if graph_ms is not None else "direct calls")
-                  + ("" if args.no_hold else ", device spin queued ahead of the start event"),
+                  + ("" if args.no_hold or not HOLD_AVAILABLE else ", device spin queued ahead of the start event"),
         "direct_calls_us_per_call": round(us_direct, 3),
         "direct_calls_frac_of_hbm_peak": round(rig.kv_bytes / (us_direct * 1e-6) / 1e9 / peak, 4),
         "kv_bytes_per_step": rig.kv_bytes,
@@ -691,7 +702,7 @@ def run_ours(args, rank, world, local_rank):
                        "together, so the dominant kernel's own rate is at least this)")
                       + ("; a bounded device spin (torch.cuda._sleep) queued ahead of the start event keeps "
                          "the GPU busy while the host submits the steps, so the region starts with the first "
-                         "step" if not args.no_hold else "; the region starts on an idle GPU"),
+                         "step" if not args.no_hold and HOLD_AVAILABLE else "; the region starts on an idle GPU"),
             "launch_ms": round(ms_per_step, 6),
             "isolated_launch_ms": round(max_iso_ms, 6),
             "isolated_launch_ms_p10_p90": [round(iso_p10, 6), round(iso_p90, 6)],
@@ -1051,8 +1062,7 @@ def run_prefill(args, rank, world, local_rank):
     torch.cuda.synchronize(device)
     sampler.mark_begin()
     if not args.no_hold:  # as in _timed_region
-        with torch.cuda.stream(stream):
-            torch.cuda._sleep(HOLD_CYCLES)
+        hold_stream(stream)
     t_start.record(stream)
     for i in range(K):
         call(i)
