@@ -44,6 +44,12 @@ CASES = [
     (4, 64, 8, 128, [0, 1, 17, 3000], 16, "persistent", 2),     # empty and 1-key sequences
     (4, 64, 4, 128, [900, 2, 0, 4000], 32, "persistent", 2),    # 16-head blocks
     (6, 64, 8, 64, [300, 40, 5000, 1, 77, 1200], 16, "persistent", 2),  # d = 64 (R = 4 per SM)
+    # the persistent grid takes as few CTAs as cover the slots in the same
+    # number of rounds: 768 slots -> 3 rounds of 256 CTAs, 1152 -> 4 of 288,
+    # 304 (just past one wave) -> 2 of 152
+    (6, 64, 8, 128, [1500, 0, 900, 33, 4096, 2000], 16, "persistent", 2),
+    (8, 64, 8, 128, [(733 * i) % 3000 + 1 for i in range(8)], 18, "persistent", 2),
+    (1, 64, 8, 128, [9000], 38, "persistent", 2),
     (6, 64, 8, 128, [5, 0, 700, 33, 4096, 16], 32, "many_waves", 1),
     (2, 96, 2, 128, [2500, 300], 200, "many_waves", 1),         # 3 head blocks of 16
 ]
