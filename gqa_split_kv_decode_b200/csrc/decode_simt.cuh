@@ -12,6 +12,13 @@
 
 namespace gqa {
 
+// L2 prefetch of `bytes` bytes at `p` (16-byte aligned, a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 template <int D, int HB, int NW, int MODE>
 __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
   static_assert(D == 64 || D == 128, "head dim");
@@ -23,6 +30,23 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = blockIdx.x, b = blockIdx.z;
   const int g = blockIdx.y / a.n_hb, hb = blockIdx.y % a.n_hb;
+  // Keys in batches of U per warp (see the key loop below).
+  constexpr int U = (HB * PER <= 8) ? 16 : (HB * PER <= 16) ? 8 : 4;
+  if (a.hint_tiles > 0 &&
+      blockIdx.x + gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z) < a.hint_ctas) {
+    // While the previous grid drains: L2 prefetch of the K and V rows of this
+    // warp's first batch, at rows from lengths read before the wait
+    // (possibly stale, so every row is checked against the cache's rows; the
+    // split is located again after the wait).
+    const Split h = locate_split<true>(a, b, slot, lane, false);
+    const long long row = h.off + h.lo + warp + (long long)lane * NW;
+    if (slot < h.n_active && lane < U && h.lo + warp + lane * NW < h.cached_hi && row >= 0 &&
+        row < a.kv_rows) {
+      const size_t at = ((size_t)row * a.h_kv + g) * D;
+      bulk_prefetch_l2(static_cast<const float*>(a.k) + at, D * 4);
+      bulk_prefetch_l2(static_cast<const float*>(a.v) + at, D * 4);
+    }
+  }
   grid_dependency_wait();
   allow_dependent_launch();
   const Split sp = locate_split(a, b, slot, lane,
@@ -61,7 +85,6 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_f32(const DecodeArgs a) {
   // batch's K and V rows are requested together, so a warp waits one memory
   // round trip per batch rather than per key, and the batch's logits share
   // one max update.
-  constexpr int U = (HB * PER <= 16) ? 8 : 4;
   for (int j0 = sp.lo + warp; j0 < sp.hi; j0 += NW * U) {
     float kr[U][PER], vr[U][PER];
 #pragma unroll

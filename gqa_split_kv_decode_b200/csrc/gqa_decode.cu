@@ -312,9 +312,15 @@ int launch_persist(const DecodeArgs& a, cudaStream_t st) {
 }
 
 template <int D, int HB, int MODE>
-int launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
+int launch_simt(DecodeArgs a, dim3 grid, cudaStream_t st) {
   constexpr int NW = 4;
-  return launch_pdl(decode_simt_f32<D, HB, NW, MODE>, grid, dim3(NW * 32), 0, st, a);
+  static std::atomic<int> per_sm[kMaxDevices];
+  auto kern = decode_simt_f32<D, HB, NW, MODE>;
+  if (a.hint_tiles > 0) {  // the grid's first wave prefetches
+    a.hint_ctas = resident_ctas(kern, NW * 32, 0, per_sm);
+    if (a.hint_ctas < 0) return GQA_ERR_CUDA;
+  }
+  return launch_pdl(kern, grid, dim3(NW * 32), 0, st, a);
 }
 
 template <int D, int MODE>
@@ -455,8 +461,9 @@ DecodeArgs make_args(const void* q, const void* k, const void* v, const int32_t*
                      long long kv_rows, const Shape& s) {
   DecodeArgs a{};
   a.kv_rows = kv_rows;
-  // the prefetch addresses are only provably inside the cache when its rows are known
-  a.hint_tiles = (s.dtype == GQA_BF16 && kv_rows >= 0) ? kHintTiles : 0;
+  // the prefetch addresses are only provably inside the cache when its rows
+  // are known; the fp32 kernel prefetches its warps' first batch of keys
+  a.hint_tiles = kv_rows < 0 ? 0 : (s.dtype == GQA_BF16 ? kHintTiles : 1);
   a.q = q;
   a.k = k;
   a.v = v;
