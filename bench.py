@@ -912,6 +912,8 @@ def run_sharded(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(device)
     sampler.mark_begin()
+    if not args.no_hold:  # as in _timed_region
+        hold_stream(stream)
     t0.record(stream)
     for i in range(K):
         call(i)
